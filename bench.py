@@ -1,0 +1,602 @@
+#!/usr/bin/env python
+"""Benchmark of the Mamba-2 SSD scan library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+
+One step = one chunked-SSD prefill pass (decay prep, chunk state, state pass, chunk scan
+with output correction) over a Mamba-2-2.7B-shaped stack of 64 independent random
+layers (batch 1, 4096 tokens, H=80, P=64, G=1, N=128, chunk 256, bf16 storage, fp32
+state).  `value` is prefill tokens/s of the whole stack: B*L / (time of one step).  The
+same run also measures the cached decode step of the 2.7B-shaped decode workload (64
+layers, ssm_state [B,80,64,128] fp32 + conv_state [B,5376,3] bf16, B in {1, 16}, 64
+steps from a state built by a 4096-token prefill) and reports it under "decode".
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and
+torch.cuda.synchronize(), timed with CUDA events on the launching stream; the step is
+captured once in a CUDA graph and replayed.  Each step reads 2.8 GB of distinct layer
+inputs, far larger than the 126 MB L2, so no flush is needed between steps.  Multi-GPU
+(torchrun): every rank runs its own replica (the scan has no data-path collective);
+rank 0 prints the max time over ranks and the summed work.
+
+--impl reference times the fp64 CPU oracle (the only reference implementation there
+is), on rank 0, each step one layer of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SSD prefill tokens/s (TFLOPS, % tensor peak); decode steps/s (GB/s, % HBM)"
+
+# prefill workload: 2.7B-shaped layer, 64-layer stack
+PF = dict(B=1, L=4096, H=80, P=64, G=1, N=128, chunk=256, layers=64, seed=2)
+# decode workload: 2.7B-shaped cache, 64 layers, 64 steps after a 4096-token prefill
+DEC = dict(H=80, P=64, G=1, N=128, K=4, layers=64, steps=64, prefix=4096, seed=4)
+
+
+# ---------------------------------------------------------------------------------------
+# work accounting (algorithmic: the inputs and outputs the method must touch)
+# ---------------------------------------------------------------------------------------
+def prefill_flops(B, L, H, P, G, N, chunk):
+    """Dense-tile flops of one prefill: per padded token 2GQN + 2HQP + 4HNP."""
+    Lp = -(-L // chunk) * chunk
+    return B * Lp * (2 * G * chunk * N + 2 * H * chunk * P + 4 * H * N * P)
+
+
+def prefill_flops_causal(B, L, H, P, G, N, chunk):
+    nc = -(-L // chunk)
+    tri = chunk * (chunk + 1)  # 2 * (Q(Q+1)/2)
+    return B * nc * (G * tri * N + H * tri * P + 4 * H * N * P * chunk)
+
+
+def chunk_scan_flops(B, L, H, P, G, N, chunk):
+    """The chunk-scan kernel's share: C.B^T once per group, the masked product, C h_prev."""
+    Lp = -(-L // chunk) * chunk
+    return B * Lp * (2 * G * chunk * N + 2 * H * chunk * P + 2 * H * N * P)
+
+
+def chunk_state_flops(B, L, H, P, G, N, chunk):
+    Lp = -(-L // chunk) * chunk
+    return B * Lp * 2 * H * N * P
+
+
+def prefill_bytes(B, L, H, P, G, N, e=2, h0=False):
+    return B * L * (2 * H * P * e + 2 * G * N * e + H * e) + (2 if h0 else 1) * B * H * P * N * 4
+
+
+def decode_bytes(B, H, P, G, N, K, e=2):
+    Cc = H * P + 2 * G * N
+    return (8 * B * H * P * N + 2 * B * Cc * (K - 1) * e + B * Cc * e + Cc * K * e + Cc * e
+            + B * H * P * e + B * H * e + 3 * H * 4)
+
+
+# ---------------------------------------------------------------------------------------
+# environment helpers
+# ---------------------------------------------------------------------------------------
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while active."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.f = None
+
+    def __enter__(self):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        try:
+            self.f.seek(0)
+            for line in open(self.f.name):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
+        finally:
+            try:
+                os.unlink(self.f.name)
+            except OSError:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [r for r in rows if r[2] > 250.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(loaded), "power_w_max": max(r[2] for r in rows)}
+
+
+def gpu_smi_id(torch):
+    """nvidia-smi -i selector of the current device (its UUID, robust to device remapping)."""
+    try:
+        u = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(torch.cuda.current_device())
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def max_over_ranks(value, world, device=None):
+    """Max of a float over all ranks (identity at world size 1)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value, world, device=None):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle timing (the cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------------------
+def oracle_layer_inputs():
+    import ssd_synth as S
+    inp = S.prefill_inputs(PF["B"], PF["L"], PF["H"], PF["P"], PF["G"], PF["N"], dtype="bf16",
+                           seed=S.layer_seed(PF["seed"], 0))
+    return {k: (v[1] if isinstance(v, tuple) else v) for k, v in inp.items()}
+
+
+def oracle_step(f):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.ssd_scan_sequential(f["x"], f["dt"], f["A_log"], f["Bm"], f["Cm"], f["D"], f["dt_bias"],
+                               f["dt_min"], f["dt_max"], None)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(min_seconds=10.0, max_reps=50):
+    import oracle
+    f = oracle_layer_inputs()
+    times = []
+    t_start = time.perf_counter()
+    while len(times) < max_reps and (time.perf_counter() - t_start) < min_seconds:
+        times.append(oracle_step(f))
+    per_layer = statistics.median(times)
+    tok_s = PF["B"] * PF["L"] / (per_layer * PF["layers"])
+    return {"value": tok_s, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": (f"fp64 sequential recurrence on 1 of the 64 layers (all {PF['L']} tokens, "
+                       f"{PF['H']} heads), {len(times)} runs, median {per_layer:.3f} s per layer; "
+                       f"stack rate = per-layer rate / 64"),
+            "host_cpu": _cpu_model(), "nproc": os.cpu_count()}
+
+
+def _cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    f = oracle_layer_inputs()
+    for _ in range(args.warmup):
+        oracle_step(f)
+    times = [oracle_step(f) for _ in range(args.steps)]
+    per_layer = statistics.mean(times)
+    value = PF["B"] * PF["L"] / (per_layer * PF["layers"])
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_layer * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.max_threads(),
+                         "kind": "oracle",
+                         "sample": "each step: fp64 sequential recurrence over 1 of the 64 layers "
+                                   "(4096 tokens, 80 heads); stack rate = per-layer rate / 64"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config():
+    return {"workload": (f"m2p7b_stack: Mamba-2-2.7B-shaped SSD prefill, batch {PF['B']}, "
+                         f"L={PF['L']}, H={PF['H']}, P={PF['P']}, G={PF['G']}, N={PF['N']}, "
+                         f"chunk {PF['chunk']}, {PF['layers']} independent random layers"),
+            "global_batch": PF["B"], "seq_len": PF["L"], "layers": PF["layers"],
+            "decode_workload": ("m2p7b_decode: 64 layers x ssm_state[B,80,64,128] fp32 + "
+                                "conv_state[B,5376,3] bf16, K=4, 64 steps after a 4096-token prefill"),
+            "l2": "inputs larger than L2 (each step reads 2.8 GB of distinct layer inputs); no flush",
+            "parallelism": "replicas (no data-path collective)"}
+
+
+# ---------------------------------------------------------------------------------------
+# GPU legs
+# ---------------------------------------------------------------------------------------
+def make_prefill_layers(torch, device, layers, rank):
+    H, P, G, N, B, L = PF["H"], PF["P"], PF["G"], PF["N"], PF["B"], PF["L"]
+    out = []
+    for layer in range(layers):
+        g = torch.Generator(device=device)
+        g.manual_seed(PF["seed"] * 1000 + layer + 100_000 * rank)
+        bf = torch.bfloat16
+        x = torch.randn((B, L, H, P), generator=g, device=device).to(bf)
+        dt = (torch.randn((B, L, H), generator=g, device=device) - 2.0).to(bf)
+        s = 1.0 / math.sqrt(N)
+        Bm = (torch.randn((B, L, G, N), generator=g, device=device) * s).to(bf)
+        Cm = (torch.randn((B, L, G, N), generator=g, device=device) * s).to(bf)
+        A_log = torch.log(torch.rand((H,), generator=g, device=device) * 15.0 + 1.0)
+        D = torch.randn((H,), generator=g, device=device)
+        dt_bias = torch.zeros((H,), device=device)
+        y = torch.empty_like(x)
+        hf = torch.empty((B, H, P, N), device=device, dtype=torch.float32)
+        out.append(dict(x=x, dt=dt, Bm=Bm, Cm=Cm, A_log=A_log, D=D, dt_bias=dt_bias, y=y, hf=hf))
+    return out
+
+
+def prefill_call(ssd, lay, ws, stream=None):
+    ssd.ssd_chunk_scan_fwd(lay["x"], lay["dt"], lay["A_log"], lay["Bm"], lay["Cm"], D=lay["D"],
+                           chunk=PF["chunk"], h0=None, dt_bias=lay["dt_bias"], dt_min=1e-3,
+                           dt_max=0.1, y=lay["y"], h_final=lay["hf"], workspace=ws, stream=stream)
+
+
+def kernel_times(torch, ssd_lib, run_eager, names):
+    """Per-kernel CUDA-event durations of one eager pass of the step.  A long sleep kernel
+    is queued first so that every launch is enqueued before the GPU reaches it: the events
+    then time the kernels, not the host."""
+    torch.cuda.synchronize()
+    ssd_lib.ssd_kernel_timer_enable(1)
+    for n in names:  # drop stale records
+        ssd_lib.ssd_kernel_timer_read(n.encode(), None, None)
+    torch.cuda._sleep(200_000_000)
+    run_eager()
+    torch.cuda.synchronize()
+    ssd_lib.ssd_kernel_timer_enable(0)
+    import ctypes
+    res = {}
+    for n in names:
+        ms = ctypes.c_double(0)
+        cnt = ctypes.c_longlong(0)
+        ssd_lib.ssd_kernel_timer_read(n.encode(), ctypes.byref(ms), ctypes.byref(cnt))
+        res[n] = (ms.value, cnt.value)
+    return res
+
+
+def bench_prefill(args, torch, ssd, device, rank, world):
+    from mamba_ssd_b200 import _lib
+    lib = _lib.lib()
+    layers = make_prefill_layers(torch, device, PF["layers"], rank)
+    B, L, H, P, G, N, Q = PF["B"], PF["L"], PF["H"], PF["P"], PF["G"], PF["N"], PF["chunk"]
+    ws = torch.empty(ssd.ssd_chunk_scan_workspace_size(B, L, H, P, G, N, Q, torch.bfloat16),
+                     device=device, dtype=torch.uint8)
+    stream = torch.cuda.Stream(device=device)
+
+    def step_eager():
+        for lay in layers:
+            prefill_call(ssd, lay, ws)
+
+    # one eager pass (sets kernel attributes before capture), then capture the step
+    with torch.cuda.stream(stream):
+        step_eager()
+    torch.cuda.synchronize()
+    n0 = lib.ssd_kernel_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step_eager()
+    launches_per_step = lib.ssd_kernel_launch_count() - n0
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_smi_id(torch)) as clocks:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    ms_max = max_over_ranks(ms, world, device)
+
+    names = ["decay_prep", "chunk_state", "state_pass", "chunk_scan"]
+    with torch.cuda.stream(stream):
+        kt = kernel_times(torch, lib, step_eager, names)
+    del graph
+    return dict(ms_total=ms_max, launches_per_step=launches_per_step, kernel_times=kt,
+                clocks=clocks.summary())
+
+
+def bench_decode(args, torch, ssd, device, rank, Bsz, steps):
+    """64-layer cached decode at batch Bsz: state built by conv + prefill over 4096 tokens,
+    then `steps` decode steps captured in one CUDA graph and timed."""
+    from mamba_ssd_b200 import _lib
+    lib = _lib.lib()
+    H, P, G, N, K = DEC["H"], DEC["P"], DEC["G"], DEC["N"], DEC["K"]
+    Cc = H * P + 2 * G * N
+    bf = torch.bfloat16
+    layers = []
+    pre_ws = torch.empty(ssd.ssd_chunk_scan_workspace_size(Bsz, DEC["prefix"], H, P, G, N, 256, bf),
+                         device=device, dtype=torch.uint8)
+    for layer in range(DEC["layers"]):
+        g = torch.Generator(device=device)
+        g.manual_seed(DEC["seed"] * 1000 + layer + 100_000 * rank)
+        bound = 1.0 / math.sqrt(K)
+        conv_w = ((torch.rand((Cc, K), generator=g, device=device) * 2 - 1) * bound).to(bf)
+        conv_b = ((torch.rand((Cc,), generator=g, device=device) * 2 - 1) * bound).to(bf)
+        A_log = torch.log(torch.rand((H,), generator=g, device=device) * 15.0 + 1.0)
+        D = torch.randn((H,), generator=g, device=device)
+        dt_bias = torch.zeros((H,), device=device)
+        scale = torch.ones(Cc, device=device)
+        scale[H * P:] = 1.0 / math.sqrt(N)
+        xbc = (torch.randn((Bsz, DEC["prefix"], Cc), generator=g, device=device) * scale).to(bf)
+        dtp = (torch.randn((Bsz, DEC["prefix"], H), generator=g, device=device) - 2.0).to(bf)
+        u, conv_state = ssd.ssd_causal_conv1d_fwd(xbc, conv_w, conv_b)
+        x = u[..., :H * P].reshape(Bsz, DEC["prefix"], H, P).contiguous()
+        Bm = u[..., H * P:H * P + G * N].reshape(Bsz, DEC["prefix"], G, N).contiguous()
+        Cm = u[..., H * P + G * N:].reshape(Bsz, DEC["prefix"], G, N).contiguous()
+        _, ssm = ssd.ssd_chunk_scan_fwd(x, dtp, A_log, Bm, Cm, D=D, chunk=256, dt_bias=dt_bias,
+                                        dt_min=1e-3, dt_max=0.1, workspace=pre_ws)
+        del xbc, dtp, u, x, Bm, Cm
+        xs = (torch.randn((steps, Bsz, Cc), generator=g, device=device) * scale).to(bf)
+        dts = (torch.randn((steps, Bsz, H), generator=g, device=device) - 2.0).to(bf)
+        y = torch.empty((steps, Bsz, H, P), device=device, dtype=bf)
+        layers.append(dict(ssm=ssm, conv=conv_state, w=conv_w, b=conv_b, A_log=A_log, D=D,
+                           dt_bias=dt_bias, xs=xs, dts=dts, y=y))
+    del pre_ws
+    ws = ssd.decode_workspace(Bsz, G, device)
+    torch.cuda.synchronize()
+
+    def run(step_range):
+        for s in step_range:
+            for lay in layers:
+                ssd.ssd_decode_step(lay["ssm"], lay["conv"], lay["xs"][s], lay["dts"][s], lay["A_log"],
+                                    lay["D"], lay["dt_bias"], lay["w"], lay["b"], H, P, G, N,
+                                    dt_min=1e-3, dt_max=0.1, y_t=lay["y"][s], workspace=ws)
+
+    stream = torch.cuda.Stream(device=device)
+    with torch.cuda.stream(stream):
+        run(range(1))
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    n0 = lib.ssd_kernel_launch_count()
+    with torch.cuda.graph(graph, stream=stream):
+        run(range(steps))
+    launches = lib.ssd_kernel_launch_count() - n0
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        graph.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    with torch.cuda.stream(stream):
+        kt = kernel_times(torch, lib, lambda: run(range(min(steps, 8))), ["decode_step"])
+    del graph
+    bytes_step = DEC["layers"] * decode_bytes(Bsz, H, P, G, N, K)
+    steps_s = steps / (ms / 1e3)
+    kms, kcnt = kt["decode_step"]
+    k_avg_s = kms / max(kcnt, 1) / 1e3
+    return {"batch": Bsz, "steps": steps, "layers": DEC["layers"], "ms": ms,
+            "steps_per_s": steps_s, "gbs": bytes_step * steps_s / 1e9,
+            "bytes_per_step": bytes_step, "launches": launches,
+            "kernel_avg_us": k_avg_s * 1e6,
+            "kernel_gbs": decode_bytes(Bsz, H, P, G, N, K) / k_avg_s / 1e9 if kcnt else None}
+
+
+def bench_e2e(args, torch, ssd, device, steps):
+    """Prefill tokens/s through the public API with host buffers: every step copies each
+    layer's inputs from pinned host memory to the device and reads y back."""
+    B, L, H, P, G, N, Q = PF["B"], PF["L"], PF["H"], PF["P"], PF["G"], PF["N"], PF["chunk"]
+    n_layers = PF["layers"]
+    dev_layers = make_prefill_layers(torch, device, 1, 0)[0]
+    host = []
+    for layer in range(n_layers):
+        g = torch.Generator()
+        g.manual_seed(PF["seed"] * 1000 + layer)
+        bf = torch.bfloat16
+        host.append(dict(
+            x=torch.randn((B, L, H, P), generator=g).to(bf).pin_memory(),
+            dt=(torch.randn((B, L, H), generator=g) - 2.0).to(bf).pin_memory(),
+            Bm=(torch.randn((B, L, G, N), generator=g) / math.sqrt(N)).to(bf).pin_memory(),
+            Cm=(torch.randn((B, L, G, N), generator=g) / math.sqrt(N)).to(bf).pin_memory(),
+            y=torch.empty((B, L, H, P), dtype=bf).pin_memory()))
+    ws = torch.empty(ssd.ssd_chunk_scan_workspace_size(B, L, H, P, G, N, Q, torch.bfloat16),
+                     device=device, dtype=torch.uint8)
+    h2d = sum(h[k].numel() * h[k].element_size() for h in host for k in ("x", "dt", "Bm", "Cm"))
+    d2h = sum(h["y"].numel() * h["y"].element_size() for h in host)
+    d = dev_layers
+
+    def step():
+        for h in host:
+            for k in ("x", "dt", "Bm", "Cm"):
+                d[k].copy_(h[k], non_blocking=True)
+            prefill_call(ssd, d, ws)
+            h["y"].copy_(d["y"], non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / steps
+    return {"value": B * L / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
+            "note": "one stream: per layer H2D of x, dt, B, C from pinned memory, prefill, D2H of y"}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    import mamba_ssd_b200 as ssd
+    from mamba_ssd_b200 import _lib
+    lib = _lib.lib()
+    peaks = load_peaks()
+
+    pf = bench_prefill(args, torch, ssd, device, rank, world)
+    B, L, H, P, G, N, Q = PF["B"], PF["L"], PF["H"], PF["P"], PF["G"], PF["N"], PF["chunk"]
+    ms_step = pf["ms_total"] / args.steps
+    tokens_all = sum_over_ranks(B * L * args.steps, world, device)
+    value = tokens_all / (pf["ms_total"] / 1e3)
+    flops_layer = prefill_flops(B, L, H, P, G, N, Q)
+    tflops = flops_layer * PF["layers"] * world / (ms_step / 1e3) / 1e12
+
+    # roofline of the dominant kernel (largest summed device time)
+    kt = pf["kernel_times"]
+    dom = max(kt, key=lambda n: kt[n][0])
+    dms, dcnt = kt[dom]
+    avg_s = dms / max(dcnt, 1) / 1e3
+    if dom in ("chunk_scan", "chunk_state"):
+        fl = (chunk_scan_flops if dom == "chunk_scan" else chunk_state_flops)(B, L, H, P, G, N, Q)
+        ach = fl / avg_s / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": f"{peaks['source']} bf16 burst"}
+    else:
+        by = prefill_bytes(B, L, H, P, G, N)
+        ach = by / avg_s / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"{peaks['source']} copy"}
+    roof["avg_launch_us"] = avg_s * 1e6
+    roof["launches_timed"] = dcnt
+    kernels = {n: {"total_ms": v[0], "launches": v[1], "avg_us": v[0] / max(v[1], 1) * 1e3}
+               for n, v in kt.items()}
+
+    decode = {}
+    if not args.no_decode:
+        for bsz in (1, 16):
+            r = bench_decode(args, torch, ssd, device, rank, bsz, DEC["steps"])
+            r["gbs_frac"] = r["gbs"] / peaks["hbm_gbs"]
+            if r.get("kernel_gbs"):
+                r["kernel_gbs_frac"] = r["kernel_gbs"] / peaks["hbm_gbs"]
+            decode[f"b{bsz}"] = r
+            torch.cuda.empty_cache()
+
+    e2e = None
+    if not args.no_e2e and rank == 0:
+        e2e = bench_e2e(args, torch, ssd, device, steps=max(1, min(args.steps, 3)))
+        torch.cuda.empty_cache()
+
+    cpu = None
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
+        cpu = cpu_baseline()
+
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": workload_config(),
+            "tflops": tflops, "tflops_frac": tflops * 1e12 / (peaks["bf16_tflops"] * 1e12) / world,
+            "flops_per_layer_dense": flops_layer,
+            "flops_per_layer_causal": prefill_flops_causal(B, L, H, P, G, N, Q),
+            "roofline": roof, "kernels": kernels, "decode": decode, "e2e": e2e,
+            "cpu_baseline": cpu, "clocks": pf["clocks"],
+            "gpu_launches": pf["launches_per_step"] * args.steps,
+            "peaks": peaks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

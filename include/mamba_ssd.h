@@ -1,0 +1,180 @@
+/*
+ * mamba_ssd.h -- C ABI of libmamba_ssd.so, the Mamba-2 state-space-duality (SSD)
+ * selective scan for NVIDIA B200 (sm_100a): chunked prefill and the O(1) cached
+ * decode step.
+ *
+ * Sources of the operations (page title and section):
+ *   "Compiler-First State Space Duality and Portable O(1) Autoregressive Caching for
+ *   Inference" (abstract): diagonal per-head dynamics, fixed-size chunking, cached
+ *   decode whose cost does not depend on the sequence length.
+ *   The article "Mamba-2状态空间模型的编译器优先实现" (bqwf.cn), cited [blog §x.y]:
+ *   §1.1 discretisation, chunking, decay mask L = tril(exp(segsum)); §1.2 the
+ *   intra-chunk contraction; §2.1 the constant-size state h in R^{H x P x N} and the
+ *   (kernel_size-1) conv cache; §2.2 the cache update (roll the conv window, set the
+ *   newest slot; ssm = ssm * A_bar + B_bar * x); §3.2 / §4.1 decay and state in fp32.
+ *
+ * The mathematics every entry point implements, for batch b, head h, group
+ * g = h / (H/G), token t:
+ *   dt_t = clip(softplus(dt[b,t,h] + dt_bias[h]), dt_min, dt_max)
+ *   h_t  = exp(dt_t * (-exp(A_log[h]))) * h_{t-1} + dt_t * x[b,t,h,:] (outer) B[b,t,g,:]
+ *   y[b,t,h,:] = h_t C[b,t,g,:] + D[h] * x[b,t,h,:]
+ * (the sign of A restored as -exp(A_log); B_bar = dt * B; y reads the state after
+ * the update at t).
+ *
+ * Conventions shared by every call:
+ *   - Every array argument is a DEVICE pointer owned by the caller.  The library
+ *     never allocates device memory, never synchronises, and enqueues all of its
+ *     work on `stream` (a cudaStream_t; NULL is the legacy default stream).  It
+ *     returns as soon as the work is enqueued.
+ *   - Arrays are dense, row-major, in exactly the index order written beside them.
+ *     Every pointer must be 16-byte aligned.  Inputs are read-only unless marked
+ *     "in/out".  Outputs must not alias inputs.
+ *   - `dtype` selects the storage type of the activation arrays: SSD_DTYPE_F32
+ *     (float) or SSD_DTYPE_BF16 (bfloat16).  Parameters and states (A_log, D,
+ *     dt_bias, h0, h_final, ssm_state) are always float32.  Accumulation and the
+ *     state recurrence are float32 in both cases.
+ *   - Arguments are validated before anything is enqueued; on any error nothing is
+ *     launched and an SSD_ERR_* code is returned.  A failed launch returns
+ *     SSD_ERR_CUDA; the CUDA error code is kept per host thread
+ *     (ssd_last_cuda_error) and a sticky CUDA error is not cleared.  No kernel traps.
+ */
+#ifndef MAMBA_SSD_H
+#define MAMBA_SSD_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every int-valued entry point. */
+#define SSD_OK 0
+#define SSD_ERR_INVALID_ARG 1  /* null/misaligned pointer, negative or inconsistent size */
+#define SSD_ERR_UNSUPPORTED 2  /* valid request outside what the kernels implement */
+#define SSD_ERR_WORKSPACE 3    /* workspace missing or smaller than the size query */
+#define SSD_ERR_CUDA 4         /* a CUDA call or kernel launch failed */
+#define SSD_ERR_TIMEOUT 5      /* a bounded device-side wait gave up */
+
+/* Storage types of activation arrays. */
+#define SSD_DTYPE_F32 0
+#define SSD_DTYPE_BF16 1
+
+/* Short English description of a status code (static storage, never NULL). */
+SSD_API const char *ssd_status_string(int status);
+
+/* The cudaError_t of the last SSD_ERR_CUDA returned on this host thread (0 if none). */
+SSD_API int ssd_last_cuda_error(void);
+
+/* Library ABI version, bumped on any signature change. */
+SSD_API int ssd_abi_version(void);
+
+/*
+ * Bytes of device workspace that ssd_chunk_scan_fwd needs for this shape (a multiple
+ * of 256; 0 when B == 0).  Returns 0 as well for shapes that
+ * ssd_chunk_scan_fwd would reject.  Pure host computation.
+ */
+SSD_API size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, int N, int chunk,
+                                     int dtype);
+
+/*
+ * Chunked SSD prefill ([blog §1.1, §1.2]; the state passing and the output
+ * correction C h_prev exp(cumsum) + D x are the plain reading of §1.1):
+ *   x        [B, L, H, P]  dtype      inputs
+ *   dt       [B, L, H]     dtype      raw step sizes (before softplus, bias and clip)
+ *   A_log    [H]           float      A = -exp(A_log)
+ *   Bm, Cm   [B, L, G, N]  dtype      input and output projections of the state
+ *   D        [H]           float      skip weight, NULL = 0
+ *   dt_bias  [H]           float      NULL = 0
+ *   dt_min, dt_max                    clip range of dt (0 and +inf disable it)
+ *   h0       [B, H, P, N]  float      initial state, NULL = zeros
+ *   y        [B, L, H, P]  dtype      output
+ *   h_final  [B, H, P, N]  float      state after token L-1 (h0 when L == 0); NULL = not written
+ *   chunk                              tokens per chunk; the last chunk may be ragged
+ *   workspace, workspace_bytes         >= ssd_chunk_scan_workspace_size(...), 256-byte
+ *                                      aligned, contents on entry irrelevant; it is
+ *                                      scratch for this call only
+ * Supported: H % G == 0, P == 64, N in {16, 32, 64, 128}, chunk in {64, 128, 256},
+ * L >= 0, B >= 0.  Other valid shapes return SSD_ERR_UNSUPPORTED.  Calls sharing a
+ * workspace must be ordered on one stream.
+ */
+SSD_API int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const void *Bm,
+                       const void *Cm, const float *D, const float *dt_bias, float dt_min,
+                       float dt_max, const float *h0, void *y, float *h_final, int B, int L,
+                       int H, int P, int G, int N, int chunk, int dtype, void *workspace,
+                       size_t workspace_bytes, void *stream);
+
+/*
+ * Bytes of device workspace that ssd_decode_step needs (a multiple of 256).  The
+ * workspace holds one arrival counter per (batch, group): it must be zero-filled once
+ * before its first use, and every completed call leaves it zero-filled again, so one
+ * zeroed workspace serves any number of consecutive calls on one stream.
+ */
+SSD_API size_t ssd_decode_workspace_size(int B, int G);
+
+/*
+ * One cached decode step for one layer ([blog §2.1, §2.2]):
+ *   ssm_state  [B, H, P, N]   float  in/out: h <- exp(dt*A) h + dt x (outer) B
+ *   conv_state [B, Cc, K-1]   dtype  in/out: the K-1 most recent raw xBC inputs,
+ *                                    oldest first; rolled by one and the newest input
+ *                                    appended
+ *   xBC_t      [B, Cc]        dtype  this token's raw conv input, channels [x | B | C],
+ *                                    Cc = H*P + 2*G*N
+ *   dt_t       [B, H]         dtype  raw step size
+ *   A_log, D, dt_bias, dt_min, dt_max   as for ssd_chunk_scan_fwd (D, dt_bias nullable)
+ *   conv_w     [Cc, K]        dtype  depthwise conv taps, tap K-1 multiplies the newest input
+ *   conv_b     [Cc]           dtype  conv bias, NULL = 0
+ *   y_t        [B, H, P]      dtype  output: y = h C + D x, with x, B, C = SiLU(conv + bias)
+ *   workspace  ssd_decode_workspace_size(B, G) bytes, zero-filled before first use
+ * Supported: H % G == 0, P % 16 == 0, N in {16, 32, 64, 128, 256}, 2 <= K <= 8.
+ * Calls sharing a workspace must be ordered on one stream.
+ */
+SSD_API int ssd_decode_step(float *ssm_state, void *conv_state, const void *xBC_t, const void *dt_t,
+                    const float *A_log, const float *D, const float *dt_bias, float dt_min,
+                    float dt_max, const void *conv_w, const void *conv_b, void *y_t, int B,
+                    int H, int P, int G, int N, int K, int dtype, void *workspace,
+                    size_t workspace_bytes, void *stream);
+
+/*
+ * Causal depthwise conv1d + bias + SiLU over a prefix, zero left padding ([blog §2.1]
+ * sliding-window conv), and the conv cache it leaves for decode:
+ *   xBC            [B, L, Cc]  dtype  raw inputs
+ *   conv_w         [Cc, K]     dtype  tap K-1 multiplies the newest input
+ *   conv_b         [Cc]        dtype  NULL = 0
+ *   out            [B, L, Cc]  dtype  SiLU(sum_k w[c,k] xBC[t-K+1+k, c] + b[c])
+ *   conv_state_out [B, Cc, K-1] dtype the last K-1 raw inputs, oldest first, zeros
+ *                                     before the start; NULL = not written
+ * Supported: 2 <= K <= 8, Cc % 8 == 0, L >= 0.
+ */
+SSD_API int ssd_causal_conv1d_fwd(const void *xBC, const void *conv_w, const void *conv_b, void *out,
+                          void *conv_state_out, int B, int L, int Cc, int K, int dtype,
+                          void *stream);
+
+/*
+ * Profiling hooks (host-side bookkeeping; no device memory is allocated).
+ *
+ * ssd_kernel_launch_count: kernels this library has enqueued in this process so far
+ * (every entry point, every host thread).
+ *
+ * ssd_kernel_timer_enable(1) makes every later kernel launch on this process record a
+ * pair of CUDA events around itself on its own stream; ssd_kernel_timer_read(name, ...)
+ * waits for the recorded events of kernel `name` ("decay_prep", "chunk_state",
+ * "state_pass", "chunk_scan", "decode_step", "causal_conv1d"), returns the summed
+ * device time in milliseconds and the number of launches timed, and forgets them.
+ * Do not enable the timer while a stream is being captured into a CUDA graph.
+ * Returns SSD_OK, SSD_ERR_INVALID_ARG for an unknown name, SSD_ERR_CUDA on an event error.
+ */
+SSD_API long long ssd_kernel_launch_count(void);
+SSD_API int ssd_kernel_timer_enable(int on);
+SSD_API int ssd_kernel_timer_read(const char *name, double *total_ms, long long *launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAMBA_SSD_H */

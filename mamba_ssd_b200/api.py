@@ -1,0 +1,144 @@
+"""Python binding of the C ABI, with the same names.  Argument marshalling only: torch
+tensors supply device memory and the current CUDA stream; every step of the SSD runs in
+the library's kernels.
+
+Shapes and dtypes follow include/mamba_ssd.h:
+  activations (x, dt, Bm, Cm, y, xBC, conv_state, conv_w, conv_b) are float32 or bfloat16,
+  all the same; A_log, D, dt_bias, h0, h_final, ssm_state are float32.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import _lib
+from ._lib import SSD_DTYPE_BF16, SSD_DTYPE_F32, check
+
+_DTYPES = {torch.float32: SSD_DTYPE_F32, torch.bfloat16: SSD_DTYPE_BF16}
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _dtype_code(t):
+    try:
+        return _DTYPES[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported activation dtype {t.dtype}") from None
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _need(t, name, dtype=None, shape=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def ssd_chunk_scan_workspace_size(B, L, H, P, G, N, chunk=256, dtype=torch.bfloat16):
+    return int(_lib.lib().ssd_chunk_scan_workspace_size(B, L, H, P, G, N, chunk, _DTYPES[dtype]))
+
+
+def ssd_chunk_scan_fwd(x, dt, A_log, Bm, Cm, D=None, chunk=256, h0=None, dt_bias=None,
+                       dt_min=0.0, dt_max=math.inf, y=None, h_final=None, workspace=None,
+                       want_h_final=True, stream=None):
+    """Chunked SSD prefill.  Returns (y, h_final); h_final is None if not wanted."""
+    Bsz, L, H, P = x.shape
+    G, N = Bm.shape[2], Bm.shape[3]
+    dt_code = _dtype_code(x)
+    _need(x, "x")
+    _need(dt, "dt", x.dtype, (Bsz, L, H))
+    _need(Bm, "Bm", x.dtype, (Bsz, L, G, N))
+    _need(Cm, "Cm", x.dtype, (Bsz, L, G, N))
+    _need(A_log, "A_log", torch.float32, (H,))
+    _need(D, "D", torch.float32, (H,))
+    _need(dt_bias, "dt_bias", torch.float32, (H,))
+    _need(h0, "h0", torch.float32, (Bsz, H, P, N))
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", x.dtype, x.shape)
+    if h_final is None and want_h_final:
+        h_final = torch.empty((Bsz, H, P, N), device=x.device, dtype=torch.float32)
+    _need(h_final, "h_final", torch.float32, (Bsz, H, P, N))
+    need = _lib.lib().ssd_chunk_scan_workspace_size(Bsz, L, H, P, G, N, chunk, dt_code)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), device=x.device, dtype=torch.uint8)
+    s = _lib.lib().ssd_chunk_scan_fwd(
+        _ptr(x), _ptr(dt), _ptr(A_log), _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(dt_bias),
+        float(dt_min), float(dt_max), _ptr(h0), _ptr(y), _ptr(h_final),
+        Bsz, L, H, P, G, N, int(chunk), dt_code, _ptr(workspace), workspace.numel(),
+        _stream(stream))
+    check(s, "ssd_chunk_scan_fwd")
+    return y, h_final
+
+
+def ssd_decode_workspace_size(B, G):
+    return int(_lib.lib().ssd_decode_workspace_size(B, G))
+
+
+def decode_workspace(B, G, device="cuda"):
+    """A zero-filled decode workspace (arrival counters), reusable across calls."""
+    return torch.zeros(max(ssd_decode_workspace_size(B, G), 256), device=device, dtype=torch.uint8)
+
+
+def ssd_decode_step(ssm_state, conv_state, xBC_t, dt_t, A_log, D, dt_bias, conv_w, conv_b,
+                    H, P, G, N, dt_min=0.0, dt_max=math.inf, y_t=None, workspace=None,
+                    stream=None):
+    """One cached decode step; updates ssm_state and conv_state in place.  Returns y_t."""
+    Bsz = ssm_state.shape[0]
+    K = conv_w.shape[1]
+    Cc = H * P + 2 * G * N
+    code = _dtype_code(xBC_t)
+    _need(ssm_state, "ssm_state", torch.float32, (Bsz, H, P, N))
+    _need(conv_state, "conv_state", xBC_t.dtype, (Bsz, Cc, K - 1))
+    _need(xBC_t, "xBC_t", None, (Bsz, Cc))
+    _need(dt_t, "dt_t", xBC_t.dtype, (Bsz, H))
+    _need(A_log, "A_log", torch.float32, (H,))
+    _need(D, "D", torch.float32, (H,))
+    _need(dt_bias, "dt_bias", torch.float32, (H,))
+    _need(conv_w, "conv_w", xBC_t.dtype, (Cc, K))
+    _need(conv_b, "conv_b", xBC_t.dtype, (Cc,))
+    if y_t is None:
+        y_t = torch.empty((Bsz, H, P), device=xBC_t.device, dtype=xBC_t.dtype)
+    _need(y_t, "y_t", xBC_t.dtype, (Bsz, H, P))
+    if workspace is None:
+        workspace = decode_workspace(Bsz, G, xBC_t.device)
+    s = _lib.lib().ssd_decode_step(
+        _ptr(ssm_state), _ptr(conv_state), _ptr(xBC_t), _ptr(dt_t), _ptr(A_log), _ptr(D),
+        _ptr(dt_bias), float(dt_min), float(dt_max), _ptr(conv_w), _ptr(conv_b), _ptr(y_t),
+        Bsz, H, P, G, N, K, code, _ptr(workspace), workspace.numel(), _stream(stream))
+    check(s, "ssd_decode_step")
+    return y_t
+
+
+def ssd_causal_conv1d_fwd(xBC, conv_w, conv_b=None, out=None, conv_state_out=None,
+                          want_state=True, stream=None):
+    """Prefix causal conv + SiLU.  Returns (out, conv_state_out)."""
+    Bsz, L, Cc = xBC.shape
+    K = conv_w.shape[1]
+    code = _dtype_code(xBC)
+    _need(xBC, "xBC")
+    _need(conv_w, "conv_w", xBC.dtype, (Cc, K))
+    _need(conv_b, "conv_b", xBC.dtype, (Cc,))
+    if out is None:
+        out = torch.empty_like(xBC)
+    if conv_state_out is None and want_state:
+        conv_state_out = torch.empty((Bsz, Cc, K - 1), device=xBC.device, dtype=xBC.dtype)
+    s = _lib.lib().ssd_causal_conv1d_fwd(
+        _ptr(xBC), _ptr(conv_w), _ptr(conv_b), _ptr(out), _ptr(conv_state_out), Bsz, L, Cc, K,
+        code, _stream(stream))
+    check(s, "ssd_causal_conv1d_fwd")
+    return out, conv_state_out

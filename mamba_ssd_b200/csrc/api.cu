@@ -1,0 +1,275 @@
+// api.cu -- the extern "C" boundary of libmamba_ssd.so: argument validation, workspace
+// carving and kernel sequencing.  Every check happens before anything is enqueued.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+// ---- profiling hooks: launch counter and optional per-kernel CUDA-event timing ----
+const char *const kKernelNames[] = {"decay_prep", "chunk_state", "state_pass",
+                                    "chunk_scan", "decode_step", "causal_conv1d"};
+enum KernelId { K_DECAY = 0, K_STATE, K_PASS, K_SCAN, K_DECODE, K_CONV, K_COUNT };
+
+std::atomic<long long> g_launches{0};
+std::atomic<int> g_timer_on{0};
+std::mutex g_timer_mu;
+std::vector<cudaEvent_t> g_event_pool;
+std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_timed[K_COUNT];
+
+cudaEvent_t pooled_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// Runs one launcher, counting it and (when the timer is on) bracketing it with events.
+template <typename F>
+cudaError_t timed_launch(KernelId id, cudaStream_t st, F &&launch) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (!g_timer_on.load(std::memory_order_relaxed)) return launch();
+    cudaEvent_t a, b;
+    {
+        std::lock_guard<std::mutex> lk(g_timer_mu);
+        a = pooled_event();
+        b = pooled_event();
+    }
+    if (!a || !b) return cudaErrorMemoryAllocation;
+    cudaEventRecord(a, st);
+    const cudaError_t e = launch();
+    cudaEventRecord(b, st);
+    std::lock_guard<std::mutex> lk(g_timer_mu);
+    g_timed[id].emplace_back(a, b);
+    return e;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool opt_aligned16(const void *p) { return p == nullptr || aligned16(p); }
+
+inline int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return SSD_OK;
+    g_last_cuda_error = (int)e;
+    return SSD_ERR_CUDA;
+}
+
+inline bool is_pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
+
+int check_dt_range(float dt_min, float dt_max) {
+    if (isnan(dt_min) || isnan(dt_max) || dt_min < 0.f || dt_min > dt_max) return SSD_ERR_INVALID_ARG;
+    return SSD_OK;
+}
+
+// Shape checks shared by the prefill size query and the call itself.
+int check_prefill_shape(int B, int L, int H, int P, int G, int N, int chunk, int dtype) {
+    if (B < 0 || L < 0 || H <= 0 || P <= 0 || G <= 0 || N <= 0 || chunk <= 0) return SSD_ERR_INVALID_ARG;
+    if (dtype != SSD_DTYPE_F32 && dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
+    if (H % G != 0) return SSD_ERR_INVALID_ARG;
+    if (P != 64) return SSD_ERR_UNSUPPORTED;
+    if (N != 16 && N != 32 && N != 64 && N != 128) return SSD_ERR_UNSUPPORTED;
+    if (chunk != 64 && chunk != 128 && chunk != 256) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+}  // namespace
+
+namespace ssd {
+
+size_t prefill_workspace_bytes(int B, int L, int H, int P, int N, int chunk) {
+    const size_t nc = (size_t)cdiv(L, chunk), Lp = nc * chunk;
+    const size_t per_tok = align_up(sizeof(float) * (size_t)B * H * Lp, 256);
+    const size_t states = align_up(sizeof(float) * (size_t)B * nc * H * P * N, 256);
+    return 2 * per_tok + states;
+}
+
+PrefillWorkspace carve_prefill_workspace(void *base, int B, int L, int H, int P, int N, int chunk) {
+    const size_t nc = (size_t)cdiv(L, chunk), Lp = nc * chunk;
+    const size_t per_tok = align_up(sizeof(float) * (size_t)B * H * Lp, 256);
+    char *p = static_cast<char *>(base);
+    PrefillWorkspace w;
+    w.dtf = reinterpret_cast<float *>(p);
+    w.acs = reinterpret_cast<float *>(p + per_tok);
+    w.states = reinterpret_cast<float *>(p + 2 * per_tok);
+    return w;
+}
+
+}  // namespace ssd
+
+extern "C" {
+
+const char *ssd_status_string(int status) {
+    switch (status) {
+        case SSD_OK: return "ok";
+        case SSD_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad size)";
+        case SSD_ERR_UNSUPPORTED: return "shape or dtype not supported by the kernels";
+        case SSD_ERR_WORKSPACE: return "workspace missing or too small";
+        case SSD_ERR_CUDA: return "CUDA error (see ssd_last_cuda_error)";
+        case SSD_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int ssd_last_cuda_error(void) { return g_last_cuda_error; }
+
+int ssd_abi_version(void) { return 1; }
+
+size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, int N, int chunk,
+                                     int dtype) {
+    if (check_prefill_shape(B, L, H, P, G, N, chunk, dtype) != SSD_OK) return 0;
+    if (B == 0) return 0;
+    return ssd::prefill_workspace_bytes(B, L, H, P, N, chunk);
+}
+
+int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const void *Bm,
+                       const void *Cm, const float *D, const float *dt_bias, float dt_min,
+                       float dt_max, const float *h0, void *y, float *h_final, int B, int L,
+                       int H, int P, int G, int N, int chunk, int dtype, void *workspace,
+                       size_t workspace_bytes, void *stream) {
+    int s = check_prefill_shape(B, L, H, P, G, N, chunk, dtype);
+    if (s != SSD_OK) return s;
+    if ((s = check_dt_range(dt_min, dt_max)) != SSD_OK) return s;
+    if (B == 0) return SSD_OK;
+    if (!A_log || !aligned16(A_log) || !opt_aligned16(D) || !opt_aligned16(dt_bias) ||
+        !opt_aligned16(h0) || !opt_aligned16(h_final))
+        return SSD_ERR_INVALID_ARG;
+    if (L > 0) {
+        if (!x || !dt || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
+        if (!aligned16(x) || !aligned16(dt) || !aligned16(Bm) || !aligned16(Cm) || !aligned16(y))
+            return SSD_ERR_INVALID_ARG;
+    }
+    const size_t need = ssd::prefill_workspace_bytes(B, L, H, P, N, chunk);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return SSD_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ssd::PrefillWorkspace ws = ssd::carve_prefill_workspace(workspace, B, L, H, P, N, chunk);
+    cudaError_t e = cudaSuccess;
+    if (L > 0) {
+        e = timed_launch(K_DECAY, st, [&] {
+            return ssd::launch_decay_prep(dtype, dt, A_log, dt_bias, dt_min, dt_max, ws.dtf, ws.acs,
+                                          B, L, H, chunk, st);
+        });
+        if (e != cudaSuccess) return cuda_status(e);
+        e = timed_launch(K_STATE, st, [&] {
+            return ssd::launch_chunk_state(dtype, x, Bm, ws.dtf, ws.acs, ws.states, B, L, H, G, N,
+                                           chunk, st);
+        });
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    e = timed_launch(K_PASS, st, [&] {
+        return ssd::launch_state_pass(ws.states, ws.acs, h0, h_final, B, L, H, P, N, chunk, st);
+    });
+    if (e != cudaSuccess) return cuda_status(e);
+    if (L > 0) {
+        e = timed_launch(K_SCAN, st, [&] {
+            return ssd::launch_chunk_scan(dtype, x, Bm, Cm, ws.dtf, ws.acs, ws.states, D, y, B, L, H,
+                                          G, N, chunk, st);
+        });
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    return SSD_OK;
+}
+
+size_t ssd_decode_workspace_size(int B, int G) {
+    if (B <= 0 || G <= 0) return 0;
+    return ssd::align_up(sizeof(unsigned) * (size_t)B * G, 256);
+}
+
+int ssd_decode_step(float *ssm_state, void *conv_state, const void *xBC_t, const void *dt_t,
+                    const float *A_log, const float *D, const float *dt_bias, float dt_min,
+                    float dt_max, const void *conv_w, const void *conv_b, void *y_t, int B,
+                    int H, int P, int G, int N, int K, int dtype, void *workspace,
+                    size_t workspace_bytes, void *stream) {
+    if (B < 0 || H <= 0 || P <= 0 || G <= 0 || N <= 0 || K <= 0) return SSD_ERR_INVALID_ARG;
+    if (dtype != SSD_DTYPE_F32 && dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
+    if (H % G != 0) return SSD_ERR_INVALID_ARG;
+    int s = check_dt_range(dt_min, dt_max);
+    if (s != SSD_OK) return s;
+    if (P % 16 != 0) return SSD_ERR_UNSUPPORTED;
+    if (!is_pow2_in(N, 16, 256)) return SSD_ERR_UNSUPPORTED;
+    if (K < 2 || K > 8) return SSD_ERR_UNSUPPORTED;
+    if (B == 0) return SSD_OK;
+    if (!ssm_state || !conv_state || !xBC_t || !dt_t || !A_log || !conv_w || !y_t)
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned16(ssm_state) || !aligned16(conv_state) || !aligned16(xBC_t) || !aligned16(dt_t) ||
+        !aligned16(A_log) || !aligned16(conv_w) || !aligned16(y_t) || !opt_aligned16(D) ||
+        !opt_aligned16(dt_bias) || !opt_aligned16(conv_b))
+        return SSD_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < ssd_decode_workspace_size(B, G) || !aligned16(workspace))
+        return SSD_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = timed_launch(K_DECODE, st, [&] {
+        return ssd::launch_decode_step(dtype, ssm_state, conv_state, xBC_t, dt_t, A_log, D, dt_bias,
+                                       dt_min, dt_max, conv_w, conv_b, y_t, B, H, P, G, N, K,
+                                       static_cast<unsigned *>(workspace), st);
+    });
+    return cuda_status(e);
+}
+
+int ssd_causal_conv1d_fwd(const void *xBC, const void *conv_w, const void *conv_b, void *out,
+                          void *conv_state_out, int B, int L, int Cc, int K, int dtype,
+                          void *stream) {
+    if (B < 0 || L < 0 || Cc <= 0 || K <= 0) return SSD_ERR_INVALID_ARG;
+    if (dtype != SSD_DTYPE_F32 && dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
+    if (K < 2 || K > 8 || Cc % 8 != 0) return SSD_ERR_UNSUPPORTED;
+    if (B == 0) return SSD_OK;
+    if (!conv_w || !aligned16(conv_w) || !opt_aligned16(conv_b) || !opt_aligned16(conv_state_out))
+        return SSD_ERR_INVALID_ARG;
+    if (L > 0 && (!xBC || !out || !aligned16(xBC) || !aligned16(out))) return SSD_ERR_INVALID_ARG;
+    if (L == 0 && !conv_state_out) return SSD_OK;
+    if (L == 0) {
+        // empty prefix: the cache is all zeros
+        const size_t bytes = (size_t)B * Cc * (K - 1) * (dtype == SSD_DTYPE_BF16 ? 2 : 4);
+        return cuda_status(cudaMemsetAsync(conv_state_out, 0, bytes, static_cast<cudaStream_t>(stream)));
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return cuda_status(timed_launch(K_CONV, st, [&] {
+        return ssd::launch_causal_conv1d(dtype, xBC, conv_w, conv_b, out, conv_state_out, B, L, Cc, K,
+                                         st);
+    }));
+}
+
+long long ssd_kernel_launch_count(void) { return g_launches.load(); }
+
+int ssd_kernel_timer_enable(int on) {
+    g_timer_on.store(on ? 1 : 0);
+    return SSD_OK;
+}
+
+int ssd_kernel_timer_read(const char *name, double *total_ms, long long *launches) {
+    if (!name) return SSD_ERR_INVALID_ARG;
+    int id = -1;
+    for (int i = 0; i < K_COUNT; ++i)
+        if (strcmp(name, kKernelNames[i]) == 0) id = i;
+    if (id < 0) return SSD_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_timer_mu);
+    double ms_sum = 0.0;
+    int status = SSD_OK;
+    for (auto &pr : g_timed[id]) {
+        float ms = 0.f;
+        cudaError_t e = cudaEventSynchronize(pr.second);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, pr.first, pr.second);
+        if (e != cudaSuccess) status = cuda_status(e);
+        ms_sum += ms;
+        g_event_pool.push_back(pr.first);
+        g_event_pool.push_back(pr.second);
+    }
+    if (total_ms) *total_ms = ms_sum;
+    if (launches) *launches = (long long)g_timed[id].size();
+    g_timed[id].clear();
+    return status;
+}
+
+}  // extern "C"

@@ -1,0 +1,60 @@
+// common.cuh -- small device helpers shared by the SSD kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mamba_ssd.h"
+
+namespace ssd {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Storage types of activations.
+template <typename T> struct Store;
+template <> struct Store<float> {
+    static __device__ __forceinline__ float load(const float *p) { return *p; }
+    static __device__ __forceinline__ float ldg(const float *p) { return __ldg(p); }
+    static __device__ __forceinline__ float from(float v) { return v; }
+};
+template <> struct Store<__nv_bfloat16> {
+    static __device__ __forceinline__ float load(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+    static __device__ __forceinline__ float ldg(const __nv_bfloat16 *p) { return __bfloat162float(__ldg(p)); }
+    static __device__ __forceinline__ __nv_bfloat16 from(float v) { return __float2bfloat16_rn(v); }
+};
+
+template <typename T> __device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// softplus(z) = log(1 + e^z), evaluated without overflow for large z.
+__device__ __forceinline__ float softplus_f(float z) {
+    return z > 20.f ? z + log1pf(expf(-z)) : log1pf(expf(z));
+}
+
+// dt = clip(softplus(dt_raw + bias), dt_min, dt_max)
+__device__ __forceinline__ float discretise_dt(float raw, float bias, float dt_min, float dt_max) {
+    return fminf(fmaxf(softplus_f(raw + bias), dt_min), dt_max);
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.f + expf(-z)); }
+
+// Inclusive warp scan (sum) of one value per lane.
+__device__ __forceinline__ float warp_inclusive_sum(float v) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        float n = __shfl_up_sync(0xffffffffu, v, o);
+        if ((threadIdx.x & 31) >= o) v += n;
+    }
+    return v;
+}
+
+__host__ __device__ constexpr inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ constexpr inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace ssd

@@ -1,0 +1,82 @@
+// decay_prep.cu -- step a1 of the chunked SSD: discretisation and the per-chunk
+// cumulative decay.
+//
+//   dt_t  = clip(softplus(dt_raw + dt_bias[h]), dt_min, dt_max)
+//   dA_t  = dt_t * (-exp(A_log[h]))                        (float32, "the decay in fp32")
+//   acs_t = sum of dA over the chunk up to and including t  (segsum building block)
+//
+// Source: "Compiler-First State Space Duality ..." blog walk-through (bqwf.cn) §1.1
+// (discretisation, chunks of 256 tokens, L = tril(exp(segsum))), §1.2 (the fused
+// softplus -> clip -> exp chain) and §4.1 (the decay must be float32).  The printed
+// exp(softplus(A_log) * dt) has lost its sign; A = -exp(A_log) is the Mamba-2 form
+// that the paper's checkpoint parity implies.
+//
+// One CTA per (chunk, batch, block of 32 heads): the chunk's dt values for 32 heads
+// are read row by row (coalesced along heads), transposed through shared memory, and
+// each warp scans one head's chunk with shuffles.  Tokens past L get dt = 0, so
+// their decay is 1 and the chunk's last cumsum is that of the last real token.
+#include "common.cuh"
+#include "launch.h"
+
+namespace ssd {
+
+template <typename T>
+__global__ void __launch_bounds__(256) decay_prep_kernel(
+    const T *__restrict__ dt, const float *__restrict__ A_log, const float *__restrict__ dt_bias,
+    float dt_min, float dt_max, float *__restrict__ dtf, float *__restrict__ acs, int L, int H,
+    int Q, int nc) {
+    extern __shared__ float sm[];  // [32][Q + 1]
+    const int c = blockIdx.x, b = blockIdx.y, hb = blockIdx.z * 32;
+    const int nh = min(32, H - hb);
+    const int ld = Q + 1;
+    for (int idx = threadIdx.x; idx < Q * nh; idx += blockDim.x) {
+        const int t = idx / nh, j = idx - t * nh, h = hb + j;
+        const int tok = c * Q + t;
+        float v = 0.f;
+        if (tok < L) {
+            const float bias = dt_bias ? dt_bias[h] : 0.f;
+            v = discretise_dt(to_f(dt[((size_t)b * L + tok) * H + h]), bias, dt_min, dt_max);
+        }
+        sm[j * ld + t] = v;
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int per = Q / 32;  // tokens per lane (Q is a multiple of 32)
+    const size_t Lp = (size_t)nc * Q;
+    for (int j = warp; j < nh; j += 8) {
+        const int h = hb + j;
+        const float A = -expf(A_log[h]);
+        const float *row = sm + j * ld + lane * per;
+        float run = 0.f;
+        for (int i = 0; i < per; ++i) run += row[i] * A;
+        float acc = warp_inclusive_sum(run) - run;  // exclusive prefix of this lane
+        const size_t base = ((size_t)b * H + h) * Lp + (size_t)c * Q + lane * per;
+        for (int i = 0; i < per; ++i) {
+            acc += row[i] * A;
+            acs[base + i] = acc;
+            dtf[base + i] = row[i];
+        }
+    }
+}
+
+cudaError_t launch_decay_prep(int dtype, const void *dt, const float *A_log, const float *dt_bias,
+                              float dt_min, float dt_max, float *dtf, float *acs, int B, int L,
+                              int H, int chunk, cudaStream_t st) {
+    const int nc = cdiv(L, chunk);
+    dim3 grid(nc, B, cdiv(H, 32));
+    const size_t smem = sizeof(float) * 32 * (chunk + 1);
+    if (dtype == SSD_DTYPE_BF16) {
+        cudaFuncSetAttribute(decay_prep_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        decay_prep_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(
+            (const __nv_bfloat16 *)dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, L, H, chunk, nc);
+    } else {
+        cudaFuncSetAttribute(decay_prep_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+        decay_prep_kernel<float><<<grid, 256, smem, st>>>((const float *)dt, A_log, dt_bias, dt_min,
+                                                          dt_max, dtf, acs, L, H, chunk, nc);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace ssd

@@ -1,0 +1,124 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every symbol that
+include/*.h declares, sizes its workspace, and rejects bad arguments before it would
+enqueue anything (so no CUDA call is reached in these tests)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from mamba_ssd_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+L = _lib.lib()
+OK, INV, UNS, WS = _lib.SSD_OK, _lib.SSD_ERR_INVALID_ARG, _lib.SSD_ERR_UNSUPPORTED, _lib.SSD_ERR_WORKSPACE
+F32, BF16 = _lib.SSD_DTYPE_F32, _lib.SSD_DTYPE_BF16
+A = 0x10000        # a fake, 16-byte aligned device address (never dereferenced here)
+MIS = 0x10002      # a misaligned one
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        names |= set(re.findall(r"SSD_API\s+[\w\s\*]+?\b(ssd_\w+)\s*\(", open(h).read()))
+    return names
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    names = declared_symbols()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+    assert names == set(_lib.SIGNATURES), "Python signature table out of sync with the header"
+
+
+def test_status_strings_and_version():
+    for s in range(6):
+        assert L.ssd_status_string(s)
+    assert L.ssd_status_string(99) == b"unknown status"
+    assert L.ssd_abi_version() >= 1
+    assert L.ssd_last_cuda_error() == 0
+
+
+def ws_bytes(B, Lx, H, P, N, chunk):
+    nc = -(-Lx // chunk)
+    per_tok = -(-4 * B * H * nc * chunk // 256) * 256
+    states = -(-4 * B * nc * H * P * N // 256) * 256
+    return 2 * per_tok + states
+
+
+@pytest.mark.parametrize("shape", [(1, 4096, 80, 64, 1, 128, 256), (8, 2048, 64, 64, 1, 128, 256),
+                                   (2, 300, 4, 64, 2, 16, 64), (1, 1, 4, 64, 1, 32, 128),
+                                   (1, 0, 4, 64, 1, 16, 256)])
+def test_prefill_workspace_size(shape):
+    B, Lx, H, P, G, N, chunk = shape
+    got = L.ssd_chunk_scan_workspace_size(B, Lx, H, P, G, N, chunk, BF16)
+    assert got == ws_bytes(B, Lx, H, P, N, chunk) and got % 256 == 0
+    assert L.ssd_chunk_scan_workspace_size(0, Lx, H, P, G, N, chunk, BF16) == 0
+    assert L.ssd_chunk_scan_workspace_size(B, Lx, H, 32, G, N, chunk, BF16) == 0   # unsupported P
+
+
+def prefill(**kw):
+    a = dict(x=A, dt=A, A_log=A, Bm=A, Cm=A, D=A, dt_bias=A, dt_min=1e-3, dt_max=0.1, h0=None,
+             y=A, h_final=A, B=1, L=64, H=4, P=64, G=1, N=16, chunk=64, dtype=BF16, ws=A,
+             ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return L.ssd_chunk_scan_fwd(a["x"], a["dt"], a["A_log"], a["Bm"], a["Cm"], a["D"],
+                                a["dt_bias"], a["dt_min"], a["dt_max"], a["h0"], a["y"],
+                                a["h_final"], a["B"], a["L"], a["H"], a["P"], a["G"], a["N"],
+                                a["chunk"], a["dtype"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(x=None), INV), (dict(Bm=None), INV), (dict(y=None), INV), (dict(A_log=None), INV),
+    (dict(x=MIS), INV), (dict(Cm=MIS), INV), (dict(h0=MIS), INV), (dict(D=MIS), INV),
+    (dict(B=-1), INV), (dict(L=-3), INV), (dict(H=0), INV), (dict(G=3), INV), (dict(dtype=7), INV),
+    (dict(dt_min=0.5, dt_max=0.1), INV), (dict(dt_min=-1.0), INV), (dict(dt_max=float("nan")), INV),
+    (dict(P=32), UNS), (dict(N=48), UNS), (dict(N=256), UNS), (dict(chunk=100), UNS),
+    (dict(chunk=512), UNS),
+    (dict(ws=None), WS), (dict(ws_bytes=1024), WS), (dict(ws=A + 16), WS),
+    (dict(B=0), OK),
+])
+def test_prefill_validation(kw, want):
+    assert prefill(**kw) == want
+
+
+def decode(**kw):
+    a = dict(ssm=A, conv=A, xbc=A, dt=A, A_log=A, D=A, dt_bias=None, dt_min=1e-3, dt_max=0.1,
+             w=A, b=A, y=A, B=1, H=80, P=64, G=1, N=128, K=4, dtype=BF16, ws=A, ws_bytes=256,
+             stream=None)
+    a.update(kw)
+    return L.ssd_decode_step(a["ssm"], a["conv"], a["xbc"], a["dt"], a["A_log"], a["D"],
+                             a["dt_bias"], a["dt_min"], a["dt_max"], a["w"], a["b"], a["y"], a["B"],
+                             a["H"], a["P"], a["G"], a["N"], a["K"], a["dtype"], a["ws"],
+                             a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(ssm=None), INV), (dict(conv=None), INV), (dict(w=None), INV), (dict(ssm=MIS), INV),
+    (dict(H=81, G=2), INV), (dict(G=0), INV), (dict(dtype=2), INV), (dict(dt_min=0.2), INV),
+    (dict(P=24), UNS), (dict(N=48), UNS), (dict(N=512), UNS), (dict(K=1), UNS), (dict(K=9), UNS),
+    (dict(ws=None), WS), (dict(ws_bytes=0), WS), (dict(B=300), WS),
+    (dict(B=0), OK),
+])
+def test_decode_validation(kw, want):
+    assert decode(**kw) == want
+
+
+def test_decode_workspace_size():
+    assert L.ssd_decode_workspace_size(1, 1) == 256
+    assert L.ssd_decode_workspace_size(16, 8) == 512
+    assert L.ssd_decode_workspace_size(0, 1) == 0
+
+
+@pytest.mark.parametrize("args,want", [
+    ((A, A, A, A, A, 1, 16, 64, 1, BF16, None), UNS),
+    ((A, A, A, A, A, 1, 16, 60, 4, BF16, None), UNS),
+    ((A, None, A, A, A, 1, 16, 64, 4, BF16, None), INV),
+    ((None, A, A, A, A, 1, 16, 64, 4, BF16, None), INV),
+    ((A, A, A, A, A, 0, 16, 64, 4, BF16, None), OK),
+    ((None, A, A, None, None, 2, 0, 64, 4, F32, None), OK),
+])
+def test_conv_validation(args, want):
+    assert L.ssd_causal_conv1d_fwd(*args) == want

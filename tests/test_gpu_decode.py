@@ -1,0 +1,148 @@
+"""GPU parity of ssd_decode_step and ssd_causal_conv1d_fwd (through the C ABI) against
+the fp64 oracle, and the cached-decode pipeline of the 2.7B-shaped decode workload:
+conv prefix + prefill over 4096 tokens, then decode steps, checked against the oracle
+and against a full-prefix recompute on the GPU."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ssd_synth as S
+from conftest import f64
+from parity import check_close, dev, host64
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import mamba_ssd_b200 as ssd
+
+
+def gpu_decode(state, prm, tok, H, P, G, N, ws=None):
+    y = ssd.ssd_decode_step(state["ssm"], state["conv"], dev(tok["xBC_t"][0]), dev(tok["dt_t"][0]),
+                            dev(prm["A_log"][0]), dev(prm["D"][0]), dev(prm["dt_bias"][0]),
+                            dev(prm["conv_w"][0]), dev(prm["conv_b"][0]), H, P, G, N,
+                            dt_min=prm["dt_min"], dt_max=prm["dt_max"], workspace=ws)
+    return y
+
+
+def _conv_params(H, P, G, N, K, dtype, seed):
+    prm = S.decode_params(H, P, G, N, K, seed=seed)
+    if dtype == "f32":
+        for k in ("conv_w", "conv_b"):
+            v = prm[k][1].astype(np.float32)
+            prm[k] = (v, v.astype(np.float64))
+    return prm
+
+
+@pytest.mark.parametrize("dtype,B,H,G,N,K", [
+    ("bf16", 1, 80, 1, 128, 4), ("bf16", 3, 8, 2, 64, 4), ("f32", 2, 4, 1, 16, 4),
+    ("f32", 1, 8, 2, 256, 3), ("bf16", 2, 6, 3, 32, 2), ("bf16", 16, 80, 1, 128, 4),
+])
+def test_decode_steps_match_oracle(dtype, B, H, G, N, K):
+    P = 64
+    prm = _conv_params(H, P, G, N, K, dtype, seed=3)
+    tok0 = S.decode_token_inputs(B, H, P, G, N, K, dtype=dtype, seed=4)
+    state = {"ssm": dev(tok0["ssm_state"][0]).clone(), "conv": dev(tok0["conv_state"][0]).clone()}
+    ref_ssm, ref_conv = tok0["ssm_state"][1], tok0["conv_state"][1]
+    ws = ssd.decode_workspace(B, G)
+    pf = f64(prm)
+    for step in range(3):  # consecutive steps reuse one workspace (counters reset)
+        tok = S.decode_token_inputs(B, H, P, G, N, K, dtype=dtype, seed=10 + step)
+        y = gpu_decode(state, prm, tok, H, P, G, N, ws)
+        torch.cuda.synchronize()
+        ft = f64(tok)
+        y_ref, ref_ssm, ref_conv = oracle.decode_step(
+            ref_ssm, ref_conv, ft["xBC_t"], ft["dt_t"], pf["A_log"], pf["D"], pf["dt_bias"],
+            pf["dt_min"], pf["dt_max"], pf["conv_w"], pf["conv_b"], H, P, G, N)
+        check_close(host64(y), y_ref, dtype, "y", f"step {step} y")
+        check_close(host64(state["ssm"]), ref_ssm, dtype, "h", f"step {step} state")
+        # the conv cache only moves raw inputs: exact
+        np.testing.assert_array_equal(host64(state["conv"]), ref_conv)
+    assert torch.count_nonzero(ws) == 0, "arrival counters must be left at zero"
+
+
+@pytest.mark.parametrize("dtype,B,L,Cc,K", [
+    ("bf16", 1, 1, 64, 4), ("bf16", 2, 2, 72, 4), ("f32", 1, 3, 16, 4), ("f32", 2, 70, 40, 3),
+    ("bf16", 1, 4096, 5376, 4), ("bf16", 3, 130, 128, 2),
+])
+def test_causal_conv_matches_oracle(dtype, B, L, Cc, K):
+    rng = np.random.default_rng(L + Cc)
+    xbc = S.to_storage(rng.standard_normal((B, L, Cc), dtype=np.float32), dtype)
+    w = S.to_storage(rng.uniform(-0.5, 0.5, (Cc, K)).astype(np.float32), dtype)
+    b = S.to_storage(rng.uniform(-0.5, 0.5, Cc).astype(np.float32), dtype)
+    out, cs = ssd.ssd_causal_conv1d_fwd(dev(xbc[0]), dev(w[0]), dev(b[0]))
+    torch.cuda.synchronize()
+    out_ref, cs_ref = oracle.causal_conv1d(xbc[1], w[1], b[1])
+    check_close(host64(out), out_ref, dtype, "y", "conv out")
+    np.testing.assert_array_equal(host64(cs), cs_ref)
+
+
+def test_conv_empty_prefix_gives_zero_cache():
+    xbc = torch.empty((2, 0, 64), device="cuda", dtype=torch.bfloat16)
+    w = torch.ones((64, 4), device="cuda", dtype=torch.bfloat16)
+    _, cs = ssd.ssd_causal_conv1d_fwd(xbc, w, None)
+    torch.cuda.synchronize()
+    assert cs.shape == (2, 64, 3) and torch.count_nonzero(cs) == 0
+
+
+def _split(u, H, P, G, N):
+    Bsz, L, _ = u.shape
+    x = u[..., :H * P].reshape(Bsz, L, H, P)
+    Bm = u[..., H * P:H * P + G * N].reshape(Bsz, L, G, N)
+    Cm = u[..., H * P + G * N:].reshape(Bsz, L, G, N)
+    return x, Bm, Cm
+
+
+@pytest.mark.parametrize("B,steps", [(1, 8), (16, 3)])
+def test_prefill_then_decode_pipeline(B, steps):
+    """2.7B-shaped cached decode on one layer: conv + prefill over 4096 tokens on the GPU,
+    then decode steps; y_t and the final state against the oracle (which rounds the conv
+    output of the prefix to bf16, the interface's storage type), and y_t against a
+    full-prefix recompute on the GPU."""
+    w = S.DECODE_WORKLOAD
+    H, P, G, N, K, L = w.H, w.P, w.G, w.N, w.K, w.prefix_len
+    Cc = H * P + 2 * G * N
+    prm = S.decode_params(H, P, G, N, K, seed=S.layer_seed(w.seed, 0))
+    seq = S.raw_xbc_sequence(B, L + steps, H, P, G, N, dtype="bf16", seed=S.layer_seed(w.seed, 500))
+    xbc_dev = dev(seq["xBC"][0])
+    dt_dev = dev(seq["dt"][0])
+    A_log, D, dt_bias = dev(prm["A_log"][0]), dev(prm["D"][0]), dev(prm["dt_bias"][0])
+    cw, cb = dev(prm["conv_w"][0]), dev(prm["conv_b"][0])
+    # GPU: prefix conv + prefill
+    u, conv_state = ssd.ssd_causal_conv1d_fwd(xbc_dev[:, :L].contiguous(), cw, cb)
+    x, Bm, Cm = (t.contiguous() for t in _split(u, H, P, G, N))
+    _, ssm = ssd.ssd_chunk_scan_fwd(x, dt_dev[:, :L].contiguous(), A_log, Bm, Cm, D=D, chunk=256,
+                                    dt_bias=dt_bias, dt_min=prm["dt_min"], dt_max=prm["dt_max"])
+    ws = ssd.decode_workspace(B, G)
+    ys = []
+    for j in range(steps):
+        t = L + j
+        y = ssd.ssd_decode_step(ssm, conv_state, xbc_dev[:, t].contiguous(), dt_dev[:, t].contiguous(),
+                                A_log, D, dt_bias, cw, cb, H, P, G, N, dt_min=prm["dt_min"],
+                                dt_max=prm["dt_max"], workspace=ws)
+        ys.append(host64(y))
+    torch.cuda.synchronize()
+    # oracle: same steps in fp64 (prefix conv output rounded to the bf16 interface)
+    pf = f64(prm)
+    xbc64, dt64 = seq["xBC"][1], seq["dt"][1]
+    u64, cs64 = oracle.causal_conv1d(xbc64[:, :L], pf["conv_w"], pf["conv_b"])
+    u64 = S.to_storage(u64, "bf16")[1]
+    xo, Bo, Co = _split(u64, H, P, G, N)
+    _, h64 = oracle.ssd_scan_sequential(xo, dt64[:, :L], pf["A_log"], Bo, Co, pf["D"],
+                                        pf["dt_bias"], pf["dt_min"], pf["dt_max"], None)
+    for j in range(steps):
+        t = L + j
+        y_ref, h64, cs64 = oracle.decode_step(h64, cs64, xbc64[:, t], dt64[:, t], pf["A_log"],
+                                              pf["D"], pf["dt_bias"], pf["dt_min"], pf["dt_max"],
+                                              pf["conv_w"], pf["conv_b"], H, P, G, N)
+        check_close(ys[j], y_ref, "bf16", "y", f"decode step {j}")
+    check_close(host64(ssm), h64, "bf16", "h", "state after decode")
+    np.testing.assert_array_equal(host64(conv_state), cs64)
+    # GPU full-prefix recompute over L + steps tokens: same outputs within bf16 tolerance
+    u2, _ = ssd.ssd_causal_conv1d_fwd(xbc_dev, cw, cb, want_state=False)
+    x2, B2, C2 = (t.contiguous() for t in _split(u2, H, P, G, N))
+    y_full, _ = ssd.ssd_chunk_scan_fwd(x2, dt_dev, A_log, B2, C2, D=D, chunk=256, dt_bias=dt_bias,
+                                       dt_min=prm["dt_min"], dt_max=prm["dt_max"], want_h_final=False)
+    yf = host64(y_full)
+    for j in range(steps):
+        check_close(ys[j], yf[:, L + j], "bf16", "y", f"recompute step {j}")
