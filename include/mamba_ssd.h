@@ -110,6 +110,14 @@ SSD_API int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log
                        size_t workspace_bytes, void *stream);
 
 /*
+ * Diagnostic: waits for `stream` to finish (this call synchronises, unlike every other
+ * entry point) and returns the status the last ssd_chunk_scan_fwd on `workspace` left
+ * there: SSD_OK, or SSD_ERR_TIMEOUT if one of its bounded device-side waits gave up (its
+ * outputs are then incomplete).  SSD_ERR_CUDA if the stream or the copy failed.
+ */
+SSD_API int ssd_chunk_scan_status(const void *workspace, void *stream);
+
+/*
  * Bytes of device workspace that ssd_decode_step needs (a multiple of 256).  The
  * workspace holds one arrival counter per (batch, group): it must be zero-filled once
  * before its first use, and every completed call leaves it zero-filled again, so one

@@ -2,6 +2,7 @@
 // carving and kernel sequencing.  Every check happens before anything is enqueued.
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <atomic>
@@ -66,6 +67,23 @@ inline int cuda_status(cudaError_t e) {
     return SSD_ERR_CUDA;
 }
 
+// Tensor-core kernels are used wherever they apply, unless SSD_PREFILL_KERNELS=simt is set in
+// the environment (then every shape runs on the float32 CUDA-core kernels).
+bool use_tensor_cores() {
+    static const bool on = [] {
+        const char *v = getenv("SSD_PREFILL_KERNELS");
+        return !(v && strcmp(v, "simt") == 0);
+    }();
+    return on;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
 inline bool is_pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
 
 int check_dt_range(float dt_min, float dt_max) {
@@ -88,11 +106,13 @@ int check_prefill_shape(int B, int L, int H, int P, int G, int N, int chunk, int
 
 namespace ssd {
 
+constexpr size_t kStatusSlot = 256;
+
 size_t prefill_workspace_bytes(int B, int L, int H, int P, int N, int chunk) {
     const size_t nc = (size_t)cdiv(L, chunk), Lp = nc * chunk;
     const size_t per_tok = align_up(sizeof(float) * (size_t)B * H * Lp, 256);
     const size_t states = align_up(sizeof(float) * (size_t)B * nc * H * P * N, 256);
-    return 2 * per_tok + states;
+    return kStatusSlot + 2 * per_tok + states;
 }
 
 PrefillWorkspace carve_prefill_workspace(void *base, int B, int L, int H, int P, int N, int chunk) {
@@ -100,6 +120,8 @@ PrefillWorkspace carve_prefill_workspace(void *base, int B, int L, int H, int P,
     const size_t per_tok = align_up(sizeof(float) * (size_t)B * H * Lp, 256);
     char *p = static_cast<char *>(base);
     PrefillWorkspace w;
+    w.status = reinterpret_cast<int *>(p);
+    p += kStatusSlot;
     w.dtf = reinterpret_cast<float *>(p);
     w.acs = reinterpret_cast<float *>(p + per_tok);
     w.states = reinterpret_cast<float *>(p + 2 * per_tok);
@@ -159,10 +181,14 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
     if (L > 0) {
         e = timed_launch(K_DECAY, st, [&] {
             return ssd::launch_decay_prep(dtype, dt, A_log, dt_bias, dt_min, dt_max, ws.dtf, ws.acs,
-                                          B, L, H, chunk, st);
+                                          ws.status, B, L, H, chunk, st);
         });
         if (e != cudaSuccess) return cuda_status(e);
+        const bool tc_state = use_tensor_cores() && ssd::chunk_state_tc_supported(dtype, P, N, chunk);
         e = timed_launch(K_STATE, st, [&] {
+            if (tc_state)
+                return ssd::launch_chunk_state_tc(x, Bm, ws.dtf, ws.acs, ws.states, ws.status, B, L, H, G,
+                                                  sm_count(), st);
             return ssd::launch_chunk_state(dtype, x, Bm, ws.dtf, ws.acs, ws.states, B, L, H, G, N,
                                            chunk, st);
         });
@@ -180,6 +206,16 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
         if (e != cudaSuccess) return cuda_status(e);
     }
     return SSD_OK;
+}
+
+int ssd_chunk_scan_status(const void *workspace, void *stream) {
+    if (!workspace) return SSD_ERR_INVALID_ARG;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(e);
+    int v = 0;
+    e = cudaMemcpy(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e);
+    return v;
 }
 
 size_t ssd_decode_workspace_size(int B, int G) {

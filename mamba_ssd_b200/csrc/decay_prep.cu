@@ -23,10 +23,12 @@ namespace ssd {
 template <typename T>
 __global__ void __launch_bounds__(256) decay_prep_kernel(
     const T *__restrict__ dt, const float *__restrict__ A_log, const float *__restrict__ dt_bias,
-    float dt_min, float dt_max, float *__restrict__ dtf, float *__restrict__ acs, int L, int H,
-    int Q, int nc) {
+    float dt_min, float dt_max, float *__restrict__ dtf, float *__restrict__ acs,
+    int *__restrict__ status, int L, int H, int Q, int nc) {
     extern __shared__ float sm[];  // [32][Q + 1]
     const int c = blockIdx.x, b = blockIdx.y, hb = blockIdx.z * 32;
+    // this call's status word starts clean (later kernels of the call may set a timeout)
+    if (status && c == 0 && b == 0 && blockIdx.z == 0 && threadIdx.x == 0) *status = SSD_OK;
     const int nh = min(32, H - hb);
     const int ld = Q + 1;
     for (int idx = threadIdx.x; idx < Q * nh; idx += blockDim.x) {
@@ -60,8 +62,8 @@ __global__ void __launch_bounds__(256) decay_prep_kernel(
 }
 
 cudaError_t launch_decay_prep(int dtype, const void *dt, const float *A_log, const float *dt_bias,
-                              float dt_min, float dt_max, float *dtf, float *acs, int B, int L,
-                              int H, int chunk, cudaStream_t st) {
+                              float dt_min, float dt_max, float *dtf, float *acs, int *status, int B,
+                              int L, int H, int chunk, cudaStream_t st) {
     const int nc = cdiv(L, chunk);
     dim3 grid(nc, B, cdiv(H, 32));
     const size_t smem = sizeof(float) * 32 * (chunk + 1);
@@ -69,12 +71,12 @@ cudaError_t launch_decay_prep(int dtype, const void *dt, const float *A_log, con
         cudaFuncSetAttribute(decay_prep_kernel<__nv_bfloat16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         decay_prep_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(
-            (const __nv_bfloat16 *)dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, L, H, chunk, nc);
+            (const __nv_bfloat16 *)dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, status, L, H, chunk, nc);
     } else {
         cudaFuncSetAttribute(decay_prep_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
         decay_prep_kernel<float><<<grid, 256, smem, st>>>((const float *)dt, A_log, dt_bias, dt_min,
-                                                          dt_max, dtf, acs, L, H, chunk, nc);
+                                                          dt_max, dtf, acs, status, L, H, chunk, nc);
     }
     return cudaGetLastError();
 }

@@ -6,13 +6,15 @@
 
 namespace ssd {
 
-// Prefill workspace layout, all float32 and 256-byte aligned:
+// Prefill workspace layout, 256-byte aligned pieces:
+//   status int32 (256-byte slot): SSD_OK, or SSD_ERR_TIMEOUT if a bounded wait gave up
 //   dtf    [B][H][Lp]          clipped dt per token (0 past the end of the sequence)
 //   acs    [B][H][Lp]          inclusive cumsum of dt*A inside each chunk
 //   states [B][nc][H][P][N]    chunk states, overwritten in place by the state each
 //                              chunk starts from (h_prev)
 // with nc = ceil(L / chunk), Lp = nc * chunk.
 struct PrefillWorkspace {
+    int *status;
     float *dtf;
     float *acs;
     float *states;
@@ -21,8 +23,14 @@ size_t prefill_workspace_bytes(int B, int L, int H, int P, int N, int chunk);
 PrefillWorkspace carve_prefill_workspace(void *base, int B, int L, int H, int P, int N, int chunk);
 
 cudaError_t launch_decay_prep(int dtype, const void *dt, const float *A_log, const float *dt_bias,
-                              float dt_min, float dt_max, float *dtf, float *acs, int B, int L,
-                              int H, int chunk, cudaStream_t st);
+                              float dt_min, float dt_max, float *dtf, float *acs, int *status, int B,
+                              int L, int H, int chunk, cudaStream_t st);
+
+// tensor-core chunk state (bf16 storage, P = 64, N = 128, chunk 256)
+bool chunk_state_tc_supported(int dtype, int P, int N, int chunk);
+cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const float *dtf, const float *acs,
+                                  float *states, int *status, int B, int L, int H, int G,
+                                  int num_sms, cudaStream_t st);
 
 cudaError_t launch_chunk_state(int dtype, const void *x, const void *Bm, const float *dtf,
                                const float *acs, float *states, int B, int L, int H, int G, int N,

@@ -45,7 +45,7 @@ def ws_bytes(B, Lx, H, P, N, chunk):
     nc = -(-Lx // chunk)
     per_tok = -(-4 * B * H * nc * chunk // 256) * 256
     states = -(-4 * B * nc * H * P * N // 256) * 256
-    return 2 * per_tok + states
+    return 256 + 2 * per_tok + states
 
 
 @pytest.mark.parametrize("shape", [(1, 4096, 80, 64, 1, 128, 256), (8, 2048, 64, 64, 1, 128, 256),
