@@ -199,7 +199,11 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
     });
     if (e != cudaSuccess) return cuda_status(e);
     if (L > 0) {
+        const bool tc_scan = use_tensor_cores() && ssd::chunk_scan_tc_supported(dtype, P, N, chunk);
         e = timed_launch(K_SCAN, st, [&] {
+            if (tc_scan)
+                return ssd::launch_chunk_scan_tc(x, Bm, Cm, ws.dtf, ws.acs, ws.states, D, y, ws.status, B, L,
+                                                 H, G, sm_count(), st);
             return ssd::launch_chunk_scan(dtype, x, Bm, Cm, ws.dtf, ws.acs, ws.states, D, y, B, L, H,
                                           G, N, chunk, st);
         });

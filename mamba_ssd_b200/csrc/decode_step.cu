@@ -13,43 +13,44 @@
 //
 // Data movement.  The fp32 state row h[b][h][p][:] (N floats) is the only large array;
 // each is read once and written once with 16-byte loads/stores, a row spread over
-// N/4 consecutive lanes, so a warp moves 512 contiguous bytes per instruction.  The
-// state loads are issued first so that their latency overlaps the conv work.
+// N/4 consecutive lanes, so a warp moves 512 contiguous bytes per instruction.  Every
+// independent load (state rows, conv windows, taps, dt) is issued before any of them is
+// used, so the kernel pays about one memory round trip rather than a chain of them.
 //
-// Work split.  One CTA per (batch, 16 consecutive state rows) -- always inside one
-// head because P % 16 == 0.  The CTA convolves its own 16 x-channels (it is their only
-// reader and writer) and all 2N B/C channels of its group, which every CTA of the group
-// needs.  Those B/C conv-cache entries may only be rolled after every CTA of the group
-// has read them: each CTA bumps a per-(batch, group) arrival counter once its reads are
-// done, and the CTA that arrives last rolls the B/C cache and resets the counter to
-// zero (no CTA ever waits, so nothing can hang).
+// Work split.  One CTA per (batch, ROWS consecutive state rows) -- always inside one head
+// because P % ROWS == 0 (ROWS = 16 at small batch for parallelism, 64 otherwise so the
+// shared B/C conv below is amortised over more state).  The CTA convolves its own ROWS
+// x-channels (it is their only reader and writer) and all 2N B/C channels of its group,
+// which every CTA of the group needs.  Those B/C conv-cache entries may only be rolled
+// after every CTA of the group has read them: each CTA bumps a per-(batch, group) arrival
+// counter once its reads are done, and the CTA that arrives last rolls the B/C cache and
+// resets the counter to zero (no CTA ever waits, so nothing can hang).
 #include "common.cuh"
 #include "launch.h"
 
 namespace ssd {
 
-constexpr int kRows = 16;      // state rows per CTA
-constexpr int kThreads = 128;  // threads per CTA
-constexpr int kMaxK = 8;
+constexpr int kDecThreads = 128;
 
-template <typename T, int N>
-__global__ void __launch_bounds__(kThreads) decode_step_kernel(
+template <typename T, int N, int K, int ROWS>
+__global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
     float *__restrict__ ssm, T *__restrict__ conv_state, const T *__restrict__ xBC_t,
     const T *__restrict__ dt_t, const float *__restrict__ A_log, const float *__restrict__ D,
     const float *__restrict__ dt_bias, float dt_min, float dt_max, const T *__restrict__ conv_w,
-    const T *__restrict__ conv_b, T *__restrict__ y_t, int H, int P, int G, int K,
+    const T *__restrict__ conv_b, T *__restrict__ y_t, int H, int P, int G,
     unsigned *__restrict__ counters) {
     constexpr int V = (N > 128) ? N / 128 : 1;  // float4 per thread per row
     constexpr int TPR = N / (4 * V);            // threads per row (<= 32, power of two)
-    constexpr int RPP = kThreads / TPR;         // rows per pass
-    constexpr int PASSES = (kRows + RPP - 1) / RPP;
+    constexpr int RPP = kDecThreads / TPR;      // rows per pass
+    constexpr int PASSES = (ROWS + RPP - 1) / RPP;
+    constexpr int BC_PER = (2 * N + kDecThreads - 1) / kDecThreads;  // B/C channels per thread
 
-    __shared__ float uB[N], uC[N], ux[kRows];
+    __shared__ float uB[N], uC[N], ux[ROWS];
     __shared__ float s_dt, s_a, s_d;
     __shared__ int s_last;
 
     const int b = blockIdx.y;
-    const int row0 = blockIdx.x * kRows;  // first (h*P + p) row of this CTA
+    const int row0 = blockIdx.x * ROWS;  // first (h*P + p) row of this CTA
     const int h = row0 / P;
     const int g = h / (H / G);
     const int HP = H * P, GN = G * N;
@@ -57,57 +58,86 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(
     const int tid = threadIdx.x;
     const int r_in_pass = tid / TPR, lane_in_row = tid % TPR;
 
-    // ---- issue the state loads first ----
+    // ---- issue every independent load first ----
     float4 st[PASSES][V];
     float *ssm_b = ssm + ((size_t)b * HP + row0) * N;
 #pragma unroll
     for (int ps = 0; ps < PASSES; ++ps) {
         const int r = ps * RPP + r_in_pass;
 #pragma unroll
-        for (int v = 0; v < V; ++v) {
-            if (r < kRows)
-                st[ps][v] = *reinterpret_cast<const float4 *>(ssm_b + (size_t)r * N +
-                                                              (v * TPR + lane_in_row) * 4);
+        for (int v = 0; v < V; ++v)
+            if (r < ROWS)
+                st[ps][v] = *reinterpret_cast<const float4 *>(ssm_b + (size_t)r * N + (v * TPR + lane_in_row) * 4);
+    }
+    // B/C channels of group g (read-only here)
+    float bc_win[BC_PER][K], bc_w[BC_PER][K], bc_bias[BC_PER];
+#pragma unroll
+    for (int q = 0; q < BC_PER; ++q) {
+        const int i = tid + q * kDecThreads;
+        if (i < 2 * N) {
+            const int cc = HP + (i < N ? g * N + i : GN + g * N + (i - N));
+            const T *cs = conv_state + ((size_t)b * Cc + cc) * (K - 1);
+#pragma unroll
+            for (int k = 0; k < K - 1; ++k) bc_win[q][k] = to_f(cs[k]);
+            bc_win[q][K - 1] = to_f(__ldg(xBC_t + (size_t)b * Cc + cc));
+#pragma unroll
+            for (int k = 0; k < K; ++k) bc_w[q][k] = to_f(__ldg(conv_w + (size_t)cc * K + k));
+            bc_bias[q] = conv_b ? to_f(__ldg(conv_b + cc)) : 0.f;
         }
     }
-
-    // ---- conv of the B and C channels of group g (read-only here) ----
-    for (int i = tid; i < 2 * N; i += kThreads) {
-        const int cc = HP + (i < N ? g * N + i : GN + g * N + (i - N));
-        const T *cs = conv_state + ((size_t)b * Cc + cc) * (K - 1);
-        const T *w = conv_w + (size_t)cc * K;
-        float acc = conv_b ? to_f(conv_b[cc]) : 0.f;
-        for (int k = 0; k < K - 1; ++k) acc = fmaf(to_f(w[k]), to_f(cs[k]), acc);
-        acc = fmaf(to_f(w[K - 1]), to_f(xBC_t[(size_t)b * Cc + cc]), acc);
-        const float u = silu_f(acc);
-        if (i < N) uB[i] = u; else uC[i - N] = u;
-    }
-    // ---- conv of this CTA's own x channels, rolled in place ----
-    if (tid < kRows) {
+    // this CTA's own x channels
+    T x_win[K];
+    float x_w[K], x_bias = 0.f;
+    if (tid < ROWS) {
         const int cc = row0 + tid;
-        T *cs = conv_state + ((size_t)b * Cc + cc) * (K - 1);
-        const T *w = conv_w + (size_t)cc * K;
-        const T newest = xBC_t[(size_t)b * Cc + cc];
-        T win[kMaxK];
-        for (int k = 0; k < K - 1; ++k) win[k] = cs[k];
-        win[K - 1] = newest;
-        float acc = conv_b ? to_f(conv_b[cc]) : 0.f;
-        for (int k = 0; k < K; ++k) acc = fmaf(to_f(w[k]), to_f(win[k]), acc);
+        const T *cs = conv_state + ((size_t)b * Cc + cc) * (K - 1);
+#pragma unroll
+        for (int k = 0; k < K - 1; ++k) x_win[k] = cs[k];
+        x_win[K - 1] = __ldg(xBC_t + (size_t)b * Cc + cc);
+#pragma unroll
+        for (int k = 0; k < K; ++k) x_w[k] = to_f(__ldg(conv_w + (size_t)cc * K + k));
+        x_bias = conv_b ? to_f(__ldg(conv_b + cc)) : 0.f;
+    }
+    float dt_raw = 0.f, alog = 0.f, dbias = 0.f, dskip = 0.f;
+    if (tid == 0) {
+        dt_raw = to_f(__ldg(dt_t + (size_t)b * H + h));
+        alog = __ldg(A_log + h);
+        dbias = dt_bias ? __ldg(dt_bias + h) : 0.f;
+        dskip = D ? __ldg(D + h) : 0.f;
+    }
+
+    // ---- conv outputs, x-channel cache roll, discretisation ----
+#pragma unroll
+    for (int q = 0; q < BC_PER; ++q) {
+        const int i = tid + q * kDecThreads;
+        if (i < 2 * N) {
+            float acc = bc_bias[q];
+#pragma unroll
+            for (int k = 0; k < K; ++k) acc = fmaf(bc_w[q][k], bc_win[q][k], acc);
+            const float u = silu_f(acc);
+            if (i < N) uB[i] = u; else uC[i - N] = u;
+        }
+    }
+    if (tid < ROWS) {
+        float acc = x_bias;
+#pragma unroll
+        for (int k = 0; k < K; ++k) acc = fmaf(x_w[k], to_f(x_win[k]), acc);
         ux[tid] = silu_f(acc);
-        for (int k = 0; k < K - 1; ++k) cs[k] = win[k + 1];
+        T *cs = conv_state + ((size_t)b * Cc + row0 + tid) * (K - 1);
+#pragma unroll
+        for (int k = 0; k < K - 1; ++k) cs[k] = x_win[k + 1];
     }
     if (tid == 0) {
-        const float dt = discretise_dt(to_f(dt_t[(size_t)b * H + h]), dt_bias ? dt_bias[h] : 0.f,
-                                       dt_min, dt_max);
+        const float dt = discretise_dt(dt_raw, dbias, dt_min, dt_max);
         s_dt = dt;
-        s_a = expf(dt * -expf(A_log[h]));
-        s_d = D ? D[h] : 0.f;
+        s_a = expf(dt * -expf(alog));
+        s_d = dskip;
     }
     __syncthreads();  // all reads of the shared B/C conv cache by this CTA are complete
 
     if (tid == 0) {
         __threadfence();
-        const unsigned ctas = (unsigned)((H / G) * P / kRows);
+        const unsigned ctas = (unsigned)((H / G) * P / ROWS);
         const unsigned prev = atomicAdd(&counters[b * G + g], 1u);
         s_last = (prev == ctas - 1);
     }
@@ -115,23 +145,27 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(
     if (s_last) {
         // every CTA of this (batch, group) has read the B/C cache: roll it
         __threadfence();
-        for (int i = tid; i < 2 * N; i += kThreads) {
-            const int cc = HP + (i < N ? g * N + i : GN + g * N + (i - N));
-            T *cs = conv_state + ((size_t)b * Cc + cc) * (K - 1);
-            for (int k = 0; k + 1 < K - 1; ++k) cs[k] = cs[k + 1];
-            cs[K - 2] = xBC_t[(size_t)b * Cc + cc];
+#pragma unroll
+        for (int q = 0; q < BC_PER; ++q) {
+            const int i = tid + q * kDecThreads;
+            if (i < 2 * N) {
+                const int cc = HP + (i < N ? g * N + i : GN + g * N + (i - N));
+                T *cs = conv_state + ((size_t)b * Cc + cc) * (K - 1);
+#pragma unroll
+                for (int k = 0; k < K - 1; ++k) cs[k] = from_f<T>(bc_win[q][k + 1]);
+            }
         }
         if (tid == 0) atomicExch(&counters[b * G + g], 0u);
     }
 
     // ---- state update and output ----
-    const float dt = s_dt, a = s_a, dskip = s_d;
+    const float dt = s_dt, a = s_a, dsk = s_d;
 #pragma unroll
     for (int ps = 0; ps < PASSES; ++ps) {
         const int r = ps * RPP + r_in_pass;
         float part = 0.f;
         float xv = 0.f;
-        if (r < kRows) {
+        if (r < ROWS) {
             xv = ux[r];
             const float dx = dt * xv;
 #pragma unroll
@@ -151,21 +185,48 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(
         }
 #pragma unroll
         for (int o = TPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o, TPR);
-        if (r < kRows && lane_in_row == 0)
-            y_t[(size_t)b * HP + row0 + r] = from_f<T>(part + dskip * xv);
+        if (r < ROWS && lane_in_row == 0) y_t[(size_t)b * HP + row0 + r] = from_f<T>(part + dsk * xv);
     }
 }
 
-template <typename T, int N>
-static cudaError_t decode_n(float *ssm, void *conv_state, const void *xBC_t, const void *dt_t,
-                            const float *A_log, const float *D, const float *dt_bias, float dt_min,
-                            float dt_max, const void *conv_w, const void *conv_b, void *y_t, int B,
-                            int H, int P, int G, int K, unsigned *counters, cudaStream_t st) {
-    dim3 grid(H * P / kRows, B);
-    decode_step_kernel<T, N><<<grid, kThreads, 0, st>>>(
+template <typename T, int N, int K, int ROWS>
+static cudaError_t decode_launch(float *ssm, void *conv_state, const void *xBC_t, const void *dt_t,
+                                 const float *A_log, const float *D, const float *dt_bias, float dt_min,
+                                 float dt_max, const void *conv_w, const void *conv_b, void *y_t,
+                                 int B, int H, int P, int G, unsigned *counters, cudaStream_t st) {
+    dim3 grid(H * P / ROWS, B);
+    decode_step_kernel<T, N, K, ROWS><<<grid, kDecThreads, 0, st>>>(
         ssm, (T *)conv_state, (const T *)xBC_t, (const T *)dt_t, A_log, D, dt_bias, dt_min, dt_max,
-        (const T *)conv_w, (const T *)conv_b, (T *)y_t, H, P, G, K, counters);
+        (const T *)conv_w, (const T *)conv_b, (T *)y_t, H, P, G, counters);
     return cudaGetLastError();
+}
+
+template <typename T, int N, int K>
+static cudaError_t decode_rows(bool wide, float *ssm, void *conv_state, const void *xBC_t, const void *dt_t,
+                               const float *A_log, const float *D, const float *dt_bias, float dt_min,
+                               float dt_max, const void *conv_w, const void *conv_b, void *y_t, int B,
+                               int H, int P, int G, unsigned *counters, cudaStream_t st) {
+    if (wide)
+        return decode_launch<T, N, K, 64>(ssm, conv_state, xBC_t, dt_t, A_log, D, dt_bias, dt_min, dt_max,
+                                          conv_w, conv_b, y_t, B, H, P, G, counters, st);
+    return decode_launch<T, N, K, 16>(ssm, conv_state, xBC_t, dt_t, A_log, D, dt_bias, dt_min, dt_max,
+                                      conv_w, conv_b, y_t, B, H, P, G, counters, st);
+}
+
+template <typename T, int N>
+static cudaError_t decode_k(int K, bool wide, float *ssm, void *conv_state, const void *xBC_t,
+                            const void *dt_t, const float *A_log, const float *D, const float *dt_bias,
+                            float dt_min, float dt_max, const void *conv_w, const void *conv_b, void *y_t,
+                            int B, int H, int P, int G, unsigned *counters, cudaStream_t st) {
+#define SSD_DK(KK)                                                                                   \
+    case KK:                                                                                         \
+        return decode_rows<T, N, KK>(wide, ssm, conv_state, xBC_t, dt_t, A_log, D, dt_bias, dt_min, \
+                                     dt_max, conv_w, conv_b, y_t, B, H, P, G, counters, st);
+    switch (K) {
+        SSD_DK(2) SSD_DK(3) SSD_DK(4) SSD_DK(5) SSD_DK(6) SSD_DK(7) SSD_DK(8)
+    }
+#undef SSD_DK
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode_step(int dtype, float *ssm_state, void *conv_state, const void *xBC_t,
@@ -173,27 +234,20 @@ cudaError_t launch_decode_step(int dtype, float *ssm_state, void *conv_state, co
                                const float *dt_bias, float dt_min, float dt_max,
                                const void *conv_w, const void *conv_b, void *y_t, int B, int H,
                                int P, int G, int N, int K, unsigned *counters, cudaStream_t st) {
-#define SSD_DEC(T, NN)                                                                          \
-    return decode_n<T, NN>(ssm_state, conv_state, xBC_t, dt_t, A_log, D, dt_bias, dt_min, dt_max, \
-                           conv_w, conv_b, y_t, B, H, P, G, K, counters, st)
+    // 64 rows per CTA once the batch gives enough CTAs; 16 otherwise
+    const bool wide = (P % 64 == 0) && (B >= 4);
+#define SSD_DN(T, NN)                                                                              \
+    case NN:                                                                                       \
+        return decode_k<T, NN>(K, wide, ssm_state, conv_state, xBC_t, dt_t, A_log, D, dt_bias,      \
+                               dt_min, dt_max, conv_w, conv_b, y_t, B, H, P, G, counters, st);
     if (dtype == SSD_DTYPE_BF16) {
-        switch (N) {
-            case 16: SSD_DEC(__nv_bfloat16, 16);
-            case 32: SSD_DEC(__nv_bfloat16, 32);
-            case 64: SSD_DEC(__nv_bfloat16, 64);
-            case 128: SSD_DEC(__nv_bfloat16, 128);
-            case 256: SSD_DEC(__nv_bfloat16, 256);
-        }
+        switch (N) { SSD_DN(__nv_bfloat16, 16) SSD_DN(__nv_bfloat16, 32) SSD_DN(__nv_bfloat16, 64)
+                     SSD_DN(__nv_bfloat16, 128) SSD_DN(__nv_bfloat16, 256) }
     } else {
-        switch (N) {
-            case 16: SSD_DEC(float, 16);
-            case 32: SSD_DEC(float, 32);
-            case 64: SSD_DEC(float, 64);
-            case 128: SSD_DEC(float, 128);
-            case 256: SSD_DEC(float, 256);
-        }
+        switch (N) { SSD_DN(float, 16) SSD_DN(float, 32) SSD_DN(float, 64) SSD_DN(float, 128)
+                     SSD_DN(float, 256) }
     }
-#undef SSD_DEC
+#undef SSD_DN
     return cudaErrorInvalidValue;
 }
 

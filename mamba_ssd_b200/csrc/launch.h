@@ -32,6 +32,12 @@ cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const float *dt
                                   float *states, int *status, int B, int L, int H, int G,
                                   int num_sms, cudaStream_t st);
 
+// tensor-core chunk scan (bf16 storage, P = 64, N = 128, chunk 256)
+bool chunk_scan_tc_supported(int dtype, int P, int N, int chunk);
+cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, const float *dtf,
+                                 const float *acs, const float *hprev, const float *D, void *y,
+                                 int *status, int B, int L, int H, int G, int num_sms, cudaStream_t st);
+
 cudaError_t launch_chunk_state(int dtype, const void *x, const void *Bm, const float *dtf,
                                const float *acs, float *states, int B, int L, int H, int G, int N,
                                int chunk, cudaStream_t st);
