@@ -508,10 +508,13 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--layers", type=int, default=PF["layers"],
+                    help="prefill stack depth (64 = the workload; smaller only for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    PF["layers"] = args.layers
     if args.impl == "reference":
         run_reference(args)
         return

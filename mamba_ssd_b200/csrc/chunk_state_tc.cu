@@ -17,8 +17,9 @@
 //
 // Structure: persistent CTAs (one per SM, 128 threads); CTA k owns a contiguous range of
 // (batch, chunk, head) items, so consecutive items share the chunk's B tile (64 KB, loaded
-// once per (batch, chunk, group)).  Per item: TMA the x tile [256 x 64] bf16 into one of two
-// stages (the next item's tile loads while this one computes), scale rows by w_s into hi
+// once per (batch, chunk, group)).  Per item: TMA the x tile [256 x 64] bf16 and bulk-copy
+// the item's dt and cumsum rows into one of two stages (the next item's data loads while
+// this one computes, so no global load sits on the critical path), scale rows by w_s into hi
 // (in place) and lo, one thread issues the 32 MMAs into one of two TMEM accumulators, and
 // the previous item's accumulator is drained to global memory meanwhile.
 #include "common.cuh"
@@ -30,7 +31,7 @@ namespace ssd {
 
 namespace cst {
 constexpr int Q = 256, P = 64, N = 128;
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;  // 8 warps: two per TMEM lane quarter
 constexpr uint32_t kTileX = Q * P * 2;  // 32 KB
 constexpr uint32_t kTileB = Q * N * 2;  // 64 KB (two 64-wide n halves)
 constexpr uint32_t kOffB = 0;
@@ -38,8 +39,10 @@ constexpr uint32_t kOffX0 = kOffB + kTileB;
 constexpr uint32_t kOffLo0 = kOffX0 + kTileX;
 constexpr uint32_t kOffX1 = kOffLo0 + kTileX;
 constexpr uint32_t kOffLo1 = kOffX1 + kTileX;
-constexpr uint32_t kOffW = kOffLo1 + kTileX;
-constexpr uint32_t kOffBar = kOffW + 2 * Q * 4;
+constexpr uint32_t kOffW = kOffLo1 + kTileX;          // w_s, 2 x 256 floats
+constexpr uint32_t kOffRows = kOffW + 2 * Q * 4;      // per stage: dt[256], acs[256]
+constexpr uint32_t kRowBytes = 2 * Q * 4;
+constexpr uint32_t kOffBar = kOffRows + 2 * kRowBytes;
 constexpr uint32_t kSmem = kOffBar + 64 + 1024;  // + slack for 1024-byte alignment
 constexpr uint32_t kTmemCols = 128;               // two 64-column fp32 accumulators
 }  // namespace cst
@@ -94,12 +97,16 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
         item_bch(j, b, c, h);
         return (b * nc + c) * G + h / hpg;
     };
-    auto issue_x = [&](int j) {  // thread 0 only
+    auto issue_x = [&](int j) {  // thread 0 only: x tile plus the item's dt and acs rows
         int b, c, h;
         item_bch(j, b, c, h);
         const int s = j & 1;
-        mbar_arrive_expect_tx(&bar_x[s], kTileX);
+        const size_t row = ((size_t)b * H + h) * Lp + (size_t)c * Q;
+        uint8_t *rows = smem + kOffRows + s * kRowBytes;
+        mbar_arrive_expect_tx(&bar_x[s], kTileX + kRowBytes);
         tma_load_3d(smem + (s ? kOffX1 : kOffX0), &tm_x, h * P, c * Q, b, &bar_x[s]);
+        bulk_load(rows, dtf + row, Q * 4, &bar_x[s]);
+        bulk_load(rows + Q * 4, acs + row, Q * 4, &bar_x[s]);
     };
     auto issue_b = [&](int j) {  // thread 0 only
         int b, c, h;
@@ -125,16 +132,18 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
         int b, c, h;
         item_bch(j, b, c, h);
         float *out = states + (((size_t)b * nc + c) * H + h) * (size_t)(P * N);
-        const int n = warp * 32 + lane;
-        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(s * 64);
+        // warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 and split the 64 columns
+        const int quarter = warp & 3, colhalf = warp >> 2;
+        const int n = quarter * 32 + lane;
+        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * 64 + colhalf * 32);
+        float v0[16], v1[16];
+        tmem_ld16(taddr, v0);
+        tmem_ld16(taddr + 16, v1);
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            float v[16];
-            tmem_ld16(taddr + q * 16, v);
-            tmem_wait_ld();
+        for (int i = 0; i < 16; ++i) out[(size_t)(colhalf * 32 + i) * N + n] = v0[i];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) out[(size_t)(q * 16 + i) * N + n] = v[i];
-        }
+        for (int i = 0; i < 16; ++i) out[(size_t)(colhalf * 32 + 16 + i) * N + n] = v1[i];
         tc_fence_before();
     };
 
@@ -171,10 +180,8 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
         ++x_done[s];
 
         // row weights w_s = dt_s exp(acs_last - acs_s) (0 past the end of the sequence)
-        int b, c, h;
-        item_bch(j, b, c, h);
-        const float *dt_row = dtf + ((size_t)b * H + h) * Lp + (size_t)c * Q;
-        const float *acs_row = acs + ((size_t)b * H + h) * Lp + (size_t)c * Q;
+        const float *dt_row = reinterpret_cast<const float *>(smem + kOffRows + s * kRowBytes);
+        const float *acs_row = dt_row + Q;
         const float a_last = acs_row[Q - 1];
         for (int r = tid; r < Q; r += kThreads) wbuf[s * Q + r] = dt_row[r] * expf(a_last - acs_row[r]);
         __syncthreads();
@@ -182,6 +189,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
         // x -> hi (in place) and lo, same swizzled positions
         uint8_t *xt = smem + (s ? kOffX1 : kOffX0);
         uint8_t *lo = smem + (s ? kOffLo1 : kOffLo0);
+#pragma unroll 4
         for (int q = tid; q < Q * 8; q += kThreads) {
             const int row = q >> 3, chunk = q & 7;
             const uint32_t off = sw128_offset(row, chunk);

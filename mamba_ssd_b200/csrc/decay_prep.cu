@@ -11,9 +11,9 @@
 // exp(softplus(A_log) * dt) has lost its sign; A = -exp(A_log) is the Mamba-2 form
 // that the paper's checkpoint parity implies.
 //
-// One CTA per (chunk, batch, block of 32 heads): the chunk's dt values for 32 heads
-// are read row by row (coalesced along heads), transposed through shared memory, and
-// each warp scans one head's chunk with shuffles.  Tokens past L get dt = 0, so
+// One CTA per (chunk, batch, block of 8 heads): the chunk's dt values for 8 heads are
+// read row by row (all loads of a thread issued together), transposed through shared
+// memory, and each of the 8 warps scans one head's chunk with shuffles.  Tokens past L get dt = 0, so
 // their decay is 1 and the chunk's last cumsum is that of the last real token.
 #include "common.cuh"
 #include "launch.h"
@@ -25,27 +25,38 @@ __global__ void __launch_bounds__(256) decay_prep_kernel(
     const T *__restrict__ dt, const float *__restrict__ A_log, const float *__restrict__ dt_bias,
     float dt_min, float dt_max, float *__restrict__ dtf, float *__restrict__ acs,
     int *__restrict__ status, int L, int H, int Q, int nc) {
-    extern __shared__ float sm[];  // [32][Q + 1]
-    const int c = blockIdx.x, b = blockIdx.y, hb = blockIdx.z * 32;
+    extern __shared__ float sm[];  // [8][Q + 1]
+    const int c = blockIdx.x, b = blockIdx.y, hb = blockIdx.z * 8;
     // this call's status word starts clean (later kernels of the call may set a timeout)
     if (status && c == 0 && b == 0 && blockIdx.z == 0 && threadIdx.x == 0) *status = SSD_OK;
-    const int nh = min(32, H - hb);
+    const int nh = min(8, H - hb);
     const int ld = Q + 1;
-    for (int idx = threadIdx.x; idx < Q * nh; idx += blockDim.x) {
-        const int t = idx / nh, j = idx - t * nh, h = hb + j;
+    // Q * 8 slots over 256 threads: at most 8 per thread (Q <= 256), loads issued together
+    constexpr int kPer = 8;
+    float raw[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int idx = threadIdx.x + i * 256;
+        const int t = idx >> 3, j = idx & 7;
         const int tok = c * Q + t;
-        float v = 0.f;
-        if (tok < L) {
-            const float bias = dt_bias ? dt_bias[h] : 0.f;
-            v = discretise_dt(to_f(dt[((size_t)b * L + tok) * H + h]), bias, dt_min, dt_max);
+        raw[i] = (t < Q && j < nh && tok < L) ? to_f(dt[((size_t)b * L + tok) * H + hb + j]) : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int idx = threadIdx.x + i * 256;
+        const int t = idx >> 3, j = idx & 7;
+        if (t < Q && j < nh) {
+            const int tok = c * Q + t;
+            float v = 0.f;
+            if (tok < L) v = discretise_dt(raw[i], dt_bias ? dt_bias[hb + j] : 0.f, dt_min, dt_max);
+            sm[j * ld + t] = v;
         }
-        sm[j * ld + t] = v;
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int per = Q / 32;  // tokens per lane (Q is a multiple of 32)
     const size_t Lp = (size_t)nc * Q;
-    for (int j = warp; j < nh; j += 8) {
+    for (int j = warp; j < nh; j += 8) {  // one head per warp
         const int h = hb + j;
         const float A = -expf(A_log[h]);
         const float *row = sm + j * ld + lane * per;
@@ -65,8 +76,8 @@ cudaError_t launch_decay_prep(int dtype, const void *dt, const float *A_log, con
                               float dt_min, float dt_max, float *dtf, float *acs, int *status, int B,
                               int L, int H, int chunk, cudaStream_t st) {
     const int nc = cdiv(L, chunk);
-    dim3 grid(nc, B, cdiv(H, 32));
-    const size_t smem = sizeof(float) * 32 * (chunk + 1);
+    dim3 grid(nc, B, cdiv(H, 8));
+    const size_t smem = sizeof(float) * 8 * (chunk + 1);
     if (dtype == SSD_DTYPE_BF16) {
         cudaFuncSetAttribute(decay_prep_kernel<__nv_bfloat16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -133,30 +133,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
         s_a = expf(dt * -expf(alog));
         s_d = dskip;
     }
-    __syncthreads();  // all reads of the shared B/C conv cache by this CTA are complete
-
-    if (tid == 0) {
-        __threadfence();
-        const unsigned ctas = (unsigned)((H / G) * P / ROWS);
-        const unsigned prev = atomicAdd(&counters[b * G + g], 1u);
-        s_last = (prev == ctas - 1);
-    }
-    __syncthreads();
-    if (s_last) {
-        // every CTA of this (batch, group) has read the B/C cache: roll it
-        __threadfence();
-#pragma unroll
-        for (int q = 0; q < BC_PER; ++q) {
-            const int i = tid + q * kDecThreads;
-            if (i < 2 * N) {
-                const int cc = HP + (i < N ? g * N + i : GN + g * N + (i - N));
-                T *cs = conv_state + ((size_t)b * Cc + cc) * (K - 1);
-#pragma unroll
-                for (int k = 0; k < K - 1; ++k) cs[k] = from_f<T>(bc_win[q][k + 1]);
-            }
-        }
-        if (tid == 0) atomicExch(&counters[b * G + g], 0u);
-    }
+    __syncthreads();  // conv outputs and dt are in shared memory; B/C cache reads are done
 
     // ---- state update and output ----
     const float dt = s_dt, a = s_a, dsk = s_d;
@@ -186,6 +163,32 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
 #pragma unroll
         for (int o = TPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o, TPR);
         if (r < ROWS && lane_in_row == 0) y_t[(size_t)b * HP + row0 + r] = from_f<T>(part + dsk * xv);
+    }
+
+    // ---- arrival: the last CTA of the (batch, group) rolls the shared B/C conv cache ----
+    // (every read of that cache by this CTA happened before the __syncthreads above)
+
+    if (tid == 0) {
+        __threadfence();
+        const unsigned ctas = (unsigned)((H / G) * P / ROWS);
+        const unsigned prev = atomicAdd(&counters[b * G + g], 1u);
+        s_last = (prev == ctas - 1);
+    }
+    __syncthreads();
+    if (s_last) {
+        // every CTA of this (batch, group) has read the B/C cache: roll it
+        __threadfence();
+#pragma unroll
+        for (int q = 0; q < BC_PER; ++q) {
+            const int i = tid + q * kDecThreads;
+            if (i < 2 * N) {
+                const int cc = HP + (i < N ? g * N + i : GN + g * N + (i - N));
+                T *cs = conv_state + ((size_t)b * Cc + cc) * (K - 1);
+#pragma unroll
+                for (int k = 0; k < K - 1; ++k) cs[k] = from_f<T>(bc_win[q][k + 1]);
+            }
+        }
+        if (tid == 0) atomicExch(&counters[b * G + g], 0u);
     }
 }
 

@@ -12,9 +12,9 @@
 //
 // Every (batch, head, state element) is an independent first-order recurrence, so
 // the grid covers B x H x P*N/4 threads, each owning one float4 of the state and
-// walking the chunks in order: fully coalesced 16-byte loads and stores, nc loads
-// in flight per thread chain.  The pass is HBM/L2 bound (it touches each chunk state
-// twice).
+// walking the chunks in order: fully coalesced 16-byte loads and stores, with the loads of
+// eight chunks issued together so the chain costs one memory round trip per eight chunks.
+// The pass is HBM/L2 bound (it touches each chunk state twice).
 #include "common.cuh"
 #include "launch.h"
 
@@ -25,6 +25,7 @@ __global__ void __launch_bounds__(256) state_pass_kernel(float *__restrict__ sta
                                                          const float *__restrict__ h0,
                                                          float *__restrict__ h_final, int H,
                                                          int PN, int nc, int Q) {
+    constexpr int kAhead = 8;  // chunk states loaded per round trip
     const int e = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
     const int h = blockIdx.y, b = blockIdx.z;
     if (e >= PN) return;
@@ -32,15 +33,27 @@ __global__ void __launch_bounds__(256) state_pass_kernel(float *__restrict__ sta
     float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
     if (h0) s = *reinterpret_cast<const float4 *>(h0 + bh * PN + e);
     const float *a_last = acs + bh * (size_t)nc * Q + (Q - 1);
-    for (int c = 0; c < nc; ++c) {
-        float4 *slot = reinterpret_cast<float4 *>(states + (((size_t)b * nc + c) * H + h) * PN + e);
-        const float4 in = *slot;
-        *slot = s;
-        const float a = expf(a_last[(size_t)c * Q]);
-        s.x = fmaf(a, s.x, in.x);
-        s.y = fmaf(a, s.y, in.y);
-        s.z = fmaf(a, s.z, in.z);
-        s.w = fmaf(a, s.w, in.w);
+    for (int c0 = 0; c0 < nc; c0 += kAhead) {
+        float4 in[kAhead];
+        float a[kAhead];
+#pragma unroll
+        for (int i = 0; i < kAhead; ++i) {
+            if (c0 + i < nc) {
+                in[i] = *reinterpret_cast<const float4 *>(states + (((size_t)b * nc + c0 + i) * H + h) * PN + e);
+                a[i] = a_last[(size_t)(c0 + i) * Q];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kAhead; ++i) {
+            if (c0 + i < nc) {
+                *reinterpret_cast<float4 *>(states + (((size_t)b * nc + c0 + i) * H + h) * PN + e) = s;
+                const float d = expf(a[i]);
+                s.x = fmaf(d, s.x, in[i].x);
+                s.y = fmaf(d, s.y, in[i].y);
+                s.z = fmaf(d, s.z, in[i].z);
+                s.w = fmaf(d, s.w, in[i].w);
+            }
+        }
     }
     if (h_final) *reinterpret_cast<float4 *>(h_final + bh * PN + e) = s;
 }
