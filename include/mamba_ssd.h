@@ -118,6 +118,40 @@ SSD_API int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log
 SSD_API int ssd_chunk_scan_status(const void *workspace, void *stream);
 
 /*
+ * ssd_chunk_scan_fwd for callers that cannot allocate device memory.  (The paper and its
+ * pages have no counterpart; this is an interface convenience of this library.)
+ *
+ * Who needs it: code that may not call cudaMalloc or any other allocating routine -- a
+ * plugin inside a host engine that owns all device memory and forbids allocations after
+ * start-up, a serving path that cannot afford the device synchronisation an allocation may
+ * cause, or a runtime whose memory budget is fixed at load time -- but still has to run the
+ * prefill, which needs scratch space.
+ *
+ * What it does: exactly ssd_chunk_scan_fwd (same arguments, same kernels, same results),
+ * except that the scratch comes from one device array of SSD_NOALLOC_SCRATCH_BYTES compiled
+ * into this library instead of a caller-provided workspace.  Every GPU that loads the
+ * library holds that array until the process exits.  Inputs and outputs are still the
+ * caller's.
+ *   - Shapes whose ssd_chunk_scan_workspace_size exceeds SSD_NOALLOC_SCRATCH_BYTES return
+ *     SSD_ERR_WORKSPACE without launching anything (48 MiB covers, for example, one
+ *     2.7B-shaped layer: batch 1, L = 4096, H = 80, P = 64, N = 128, chunk 256).
+ *   - The first call on each device looks up the array's device address on that device (the
+ *     device must be current); make that first call before any stream capture.
+ *   - Every call uses the same array and leaves its contents behind.  Calls that may overlap
+ *     on the GPU (different streams, different host threads without ordering) race on it and
+ *     corrupt each other's results; order them on one stream.  Nothing in the array has to be
+ *     zeroed by the caller.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define SSD_NOALLOC_SCRATCH_BYTES (48u * 1024u * 1024u)
+SSD_API int ssd_chunk_scan_fwd_noalloc(const void *x, const void *dt, const float *A_log,
+                                       const void *Bm, const void *Cm, const float *D,
+                                       const float *dt_bias, float dt_min, float dt_max,
+                                       const float *h0, void *y, float *h_final, int B, int L,
+                                       int H, int P, int G, int N, int chunk, int dtype,
+                                       void *stream);
+
+/*
  * Bytes of device workspace that ssd_decode_step needs (a multiple of 256).  The
  * workspace holds one arrival counter per (batch, group): it must be zero-filled once
  * before its first use, and every completed call leaves it zero-filled again, so one

@@ -19,6 +19,7 @@ SSD_ERR_CUDA = 4
 SSD_ERR_TIMEOUT = 5
 SSD_DTYPE_F32 = 0
 SSD_DTYPE_BF16 = 1
+SSD_NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024
 
 # name -> (restype, argtypes); must match include/mamba_ssd.h
 _vp, _fp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -30,6 +31,8 @@ SIGNATURES = {
     "ssd_chunk_scan_fwd": (_i, [_vp, _vp, _fp, _vp, _vp, _fp, _fp, _f, _f, _fp, _vp, _fp]
                            + [_i] * 8 + [_vp, _sz, _vp]),
     "ssd_chunk_scan_status": (_i, [_vp, _vp]),
+    "ssd_chunk_scan_fwd_noalloc": (_i, [_vp, _vp, _fp, _vp, _vp, _fp, _fp, _f, _f, _fp, _vp, _fp]
+                                   + [_i] * 8 + [_vp]),
     "ssd_decode_workspace_size": (_sz, [_i, _i]),
     "ssd_decode_step": (_i, [_fp, _vp, _vp, _vp, _fp, _fp, _fp, _f, _f, _vp, _vp, _vp]
                         + [_i] * 7 + [_vp, _sz, _vp]),

@@ -85,6 +85,36 @@ def ssd_chunk_scan_fwd(x, dt, A_log, Bm, Cm, D=None, chunk=256, h0=None, dt_bias
     return y, h_final
 
 
+def ssd_chunk_scan_fwd_noalloc(x, dt, A_log, Bm, Cm, D=None, chunk=256, h0=None, dt_bias=None,
+                               dt_min=0.0, dt_max=math.inf, y=None, h_final=None, stream=None):
+    """ssd_chunk_scan_fwd whose scratch is the library's built-in device array (no workspace
+    argument; for callers that cannot allocate).  Outputs y and h_final are still supplied by
+    the caller, or allocated here by torch when omitted.  Returns (y, h_final)."""
+    Bsz, L, H, P = x.shape
+    G, N = Bm.shape[2], Bm.shape[3]
+    code = _dtype_code(x)
+    _need(x, "x")
+    _need(dt, "dt", x.dtype, (Bsz, L, H))
+    _need(Bm, "Bm", x.dtype, (Bsz, L, G, N))
+    _need(Cm, "Cm", x.dtype, (Bsz, L, G, N))
+    _need(A_log, "A_log", torch.float32, (H,))
+    _need(D, "D", torch.float32, (H,))
+    _need(dt_bias, "dt_bias", torch.float32, (H,))
+    _need(h0, "h0", torch.float32, (Bsz, H, P, N))
+    if y is None:
+        y = torch.empty_like(x)
+    if h_final is None:
+        h_final = torch.empty((Bsz, H, P, N), device=x.device, dtype=torch.float32)
+    _need(y, "y", x.dtype, x.shape)
+    _need(h_final, "h_final", torch.float32, (Bsz, H, P, N))
+    s = _lib.lib().ssd_chunk_scan_fwd_noalloc(
+        _ptr(x), _ptr(dt), _ptr(A_log), _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(dt_bias),
+        float(dt_min), float(dt_max), _ptr(h0), _ptr(y), _ptr(h_final),
+        Bsz, L, H, P, G, N, int(chunk), code, _stream(stream))
+    check(s, "ssd_chunk_scan_fwd_noalloc")
+    return y, h_final
+
+
 def ssd_decode_workspace_size(B, G):
     return int(_lib.lib().ssd_decode_workspace_size(B, G))
 

@@ -1,0 +1,57 @@
+"""ssd_chunk_scan_fwd_noalloc, the prefill variant whose scratch is the library's built-in
+device array, for callers that cannot allocate device memory (engines that own all device
+memory, latency-critical paths that must not trigger an allocation).
+
+Called through the C ABI, it must give the same y and h_final as ssd_chunk_scan_fwd on the
+same inputs, within the parity tolerances of tests/parity.py, on two calls in a row (the
+second on different inputs, so stale scratch contents must not matter), and must refuse a
+shape whose scratch would not fit.  This file is collected last on purpose.
+"""
+import numpy as np
+import pytest
+import torch
+
+import ssd_synth as S
+from parity import check_close, dev, host64
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import mamba_ssd_b200 as ssd
+    from mamba_ssd_b200 import _lib
+
+
+def _both(inp, chunk):
+    args = (dev(inp["x"][0]), dev(inp["dt"][0]), dev(inp["A_log"][0]), dev(inp["Bm"][0]),
+            dev(inp["Cm"][0]))
+    kw = dict(D=dev(inp["D"][0]), chunk=chunk, h0=None if inp["h0"] is None else dev(inp["h0"][0]),
+              dt_bias=dev(inp["dt_bias"][0]), dt_min=inp["dt_min"], dt_max=inp["dt_max"])
+    y_ref, h_ref = ssd.ssd_chunk_scan_fwd(*args, **kw)
+    y, h = ssd.ssd_chunk_scan_fwd_noalloc(*args, **kw)
+    torch.cuda.synchronize()
+    return host64(y), host64(h), host64(y_ref), host64(h_ref)
+
+
+@pytest.mark.parametrize("dtype,B,L,H,N,chunk,h0", [
+    ("bf16", 1, 4096, 80, 128, 256, False),   # a 2.7B-shaped layer: the largest that fits
+    ("f32", 2, 700, 4, 16, 128, True),
+])
+def test_noalloc_matches_workspace_entry_twice(dtype, B, L, H, N, chunk, h0):
+    for call in range(2):
+        inp = S.prefill_inputs(B, L, H, 64, 1, N, dtype=dtype, seed=40 + call, h0=h0)
+        y, h, y_ref, h_ref = _both(inp, chunk)
+        check_close(y, y_ref, dtype, "y", f"noalloc call {call} y")
+        check_close(h, h_ref, dtype, "h", f"noalloc call {call} h_final")
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    B, L, H, P, G, N, chunk = 1, 8192, 80, 64, 1, 128, 256
+    need = _lib.lib().ssd_chunk_scan_workspace_size(B, L, H, P, G, N, chunk, _lib.SSD_DTYPE_BF16)
+    assert need > _lib.SSD_NOALLOC_SCRATCH_BYTES
+    x = torch.empty((B, L, H, P), device="cuda", dtype=torch.bfloat16)
+    dt = torch.empty((B, L, H), device="cuda", dtype=torch.bfloat16)
+    Bm = torch.empty((B, L, G, N), device="cuda", dtype=torch.bfloat16)
+    A_log = torch.zeros(H, device="cuda")
+    with pytest.raises(_lib.SSDError) as err:
+        ssd.ssd_chunk_scan_fwd_noalloc(x, dt, A_log, Bm, Bm)
+    assert err.value.status == _lib.SSD_ERR_WORKSPACE
