@@ -134,7 +134,7 @@ SSD_API int ssd_chunk_scan_status(const void *workspace, void *stream);
  * caller's.
  *   - Shapes whose ssd_chunk_scan_workspace_size exceeds SSD_NOALLOC_SCRATCH_BYTES return
  *     SSD_ERR_WORKSPACE without launching anything (48 MiB covers, for example, one
- *     2.7B-shaped layer: batch 1, L = 4096, H = 80, P = 64, N = 128, chunk 256).
+ *     130M-shaped layer: batch 1, L = 4096, H = 24, P = 64, N = 128, bf16).
  *   - The first call on each device looks up the array's device address on that device (the
  *     device must be current); make that first call before any stream capture.
  *   - Every call uses the same array and leaves its contents behind.  Calls that may overlap

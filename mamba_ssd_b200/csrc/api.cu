@@ -108,16 +108,19 @@ namespace ssd {
 
 constexpr size_t kStatusSlot = 256;
 
-size_t prefill_workspace_bytes(int B, int L, int H, int P, int N, int chunk) {
-    const size_t nc = (size_t)cdiv(L, chunk), Lp = nc * chunk;
+size_t prefill_workspace_bytes(int B, int L, int H, int P, int N, int block, bool transposed_bf16) {
+    const size_t nb = (size_t)cdiv(L, block), Lp = nb * block;
     const size_t per_tok = align_up(sizeof(float) * (size_t)B * H * Lp, 256);
-    const size_t states = align_up(sizeof(float) * (size_t)B * nc * H * P * N, 256);
-    return kStatusSlot + 2 * per_tok + states;
+    const size_t states = align_up(sizeof(float) * (size_t)B * nb * H * P * N, 256);
+    const size_t hT = transposed_bf16 ? align_up(2 * (size_t)B * nb * H * P * N, 256) : 0;
+    return kStatusSlot + 2 * per_tok + states + hT;
 }
 
-PrefillWorkspace carve_prefill_workspace(void *base, int B, int L, int H, int P, int N, int chunk) {
-    const size_t nc = (size_t)cdiv(L, chunk), Lp = nc * chunk;
+PrefillWorkspace carve_prefill_workspace(void *base, int B, int L, int H, int P, int N, int block,
+                                         bool transposed_bf16) {
+    const size_t nb = (size_t)cdiv(L, block), Lp = nb * block;
     const size_t per_tok = align_up(sizeof(float) * (size_t)B * H * Lp, 256);
+    const size_t states = align_up(sizeof(float) * (size_t)B * nb * H * P * N, 256);
     char *p = static_cast<char *>(base);
     PrefillWorkspace w;
     w.status = reinterpret_cast<int *>(p);
@@ -125,7 +128,19 @@ PrefillWorkspace carve_prefill_workspace(void *base, int B, int L, int H, int P,
     w.dtf = reinterpret_cast<float *>(p);
     w.acs = reinterpret_cast<float *>(p + per_tok);
     w.states = reinterpret_cast<float *>(p + 2 * per_tok);
+    w.hT = transposed_bf16 ? reinterpret_cast<__nv_bfloat16 *>(p + 2 * per_tok + states) : nullptr;
     return w;
+}
+
+// Bytes a prefill needs: the larger of the layouts its shape may run with, so that a
+// workspace sized by the query serves either path.
+size_t prefill_query_bytes(int B, int L, int H, int P, int N, int chunk, int dtype) {
+    size_t need = prefill_workspace_bytes(B, L, H, P, N, chunk, false);
+    if (prefill_tc_supported(dtype, P, N)) {
+        const size_t tc = prefill_workspace_bytes(B, L, H, P, N, kTcBlock, true);
+        if (tc > need) need = tc;
+    }
+    return need;
 }
 
 }  // namespace ssd
@@ -152,7 +167,7 @@ size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, int N, i
                                      int dtype) {
     if (check_prefill_shape(B, L, H, P, G, N, chunk, dtype) != SSD_OK) return 0;
     if (B == 0) return 0;
-    return ssd::prefill_workspace_bytes(B, L, H, P, N, chunk);
+    return ssd::prefill_query_bytes(B, L, H, P, N, chunk, dtype);
 }
 
 int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const void *Bm,
@@ -172,25 +187,50 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
         if (!aligned16(x) || !aligned16(dt) || !aligned16(Bm) || !aligned16(Cm) || !aligned16(y))
             return SSD_ERR_INVALID_ARG;
     }
-    const size_t need = ssd::prefill_workspace_bytes(B, L, H, P, N, chunk);
+    const size_t need = ssd::prefill_query_bytes(B, L, H, P, N, chunk, dtype);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return SSD_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    ssd::PrefillWorkspace ws = ssd::carve_prefill_workspace(workspace, B, L, H, P, N, chunk);
     cudaError_t e = cudaSuccess;
+    if (use_tensor_cores() && ssd::prefill_tc_supported(dtype, P, N)) {
+        // tensor-core path: 128-token blocks, block states in fp32, h_prev^T in bf16
+        const int blk = ssd::kTcBlock;
+        ssd::PrefillWorkspace ws = ssd::carve_prefill_workspace(workspace, B, L, H, P, N, blk, true);
+        if (L > 0) {
+            e = timed_launch(K_DECAY, st, [&] {
+                return ssd::launch_decay_prep(dtype, dt, A_log, dt_bias, dt_min, dt_max, ws.dtf, ws.acs,
+                                              ws.status, B, L, H, blk, true, st);
+            });
+            if (e != cudaSuccess) return cuda_status(e);
+            e = timed_launch(K_STATE, st, [&] {
+                return ssd::launch_chunk_state_tc(x, Bm, ws.dtf, ws.acs, ws.states, ws.status, B, L, H, G,
+                                                  sm_count(), st);
+            });
+            if (e != cudaSuccess) return cuda_status(e);
+        }
+        e = timed_launch(K_PASS, st, [&] {
+            return ssd::launch_state_pass_t(ws.states, ws.acs, h0, h_final, ws.hT, B, L, H, P, N, blk, st);
+        });
+        if (e != cudaSuccess) return cuda_status(e);
+        if (L > 0) {
+            e = timed_launch(K_SCAN, st, [&] {
+                return ssd::launch_chunk_scan_tc(x, Bm, Cm, ws.dtf, ws.acs, ws.hT, D, y, ws.status, B, L, H, G,
+                                                 sm_count(), st);
+            });
+            if (e != cudaSuccess) return cuda_status(e);
+        }
+        return SSD_OK;
+    }
+    // CUDA-core path: the caller's chunk, fp32 throughout
+    ssd::PrefillWorkspace ws = ssd::carve_prefill_workspace(workspace, B, L, H, P, N, chunk, false);
     if (L > 0) {
         e = timed_launch(K_DECAY, st, [&] {
             return ssd::launch_decay_prep(dtype, dt, A_log, dt_bias, dt_min, dt_max, ws.dtf, ws.acs,
-                                          ws.status, B, L, H, chunk, st);
+                                          ws.status, B, L, H, chunk, false, st);
         });
         if (e != cudaSuccess) return cuda_status(e);
-        const bool tc_state = use_tensor_cores() && ssd::chunk_state_tc_supported(dtype, P, N, chunk);
         e = timed_launch(K_STATE, st, [&] {
-            if (tc_state)
-                return ssd::launch_chunk_state_tc(x, Bm, ws.dtf, ws.acs, ws.states, ws.status, B, L, H, G,
-                                                  sm_count(), st);
-            return ssd::launch_chunk_state(dtype, x, Bm, ws.dtf, ws.acs, ws.states, B, L, H, G, N,
-                                           chunk, st);
+            return ssd::launch_chunk_state(dtype, x, Bm, ws.dtf, ws.acs, ws.states, B, L, H, G, N, chunk, st);
         });
         if (e != cudaSuccess) return cuda_status(e);
     }
@@ -199,13 +239,9 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
     });
     if (e != cudaSuccess) return cuda_status(e);
     if (L > 0) {
-        const bool tc_scan = use_tensor_cores() && ssd::chunk_scan_tc_supported(dtype, P, N, chunk);
         e = timed_launch(K_SCAN, st, [&] {
-            if (tc_scan)
-                return ssd::launch_chunk_scan_tc(x, Bm, Cm, ws.dtf, ws.acs, ws.states, D, y, ws.status, B, L,
-                                                 H, G, sm_count(), st);
-            return ssd::launch_chunk_scan(dtype, x, Bm, Cm, ws.dtf, ws.acs, ws.states, D, y, B, L, H,
-                                          G, N, chunk, st);
+            return ssd::launch_chunk_scan(dtype, x, Bm, Cm, ws.dtf, ws.acs, ws.states, D, y, B, L, H, G, N,
+                                          chunk, st);
         });
         if (e != cudaSuccess) return cuda_status(e);
     }

@@ -1,27 +1,30 @@
-// chunk_state_tc.cu -- step a3 on the tcgen05 tensor cores (bf16 storage, P = 64, N = 128,
-// chunk 256):
+// chunk_state_tc.cu -- step a3 on the tcgen05 tensor cores (bf16 storage, P = 64, N = 128):
 //
-//   S_c[p][n] = sum_{s in chunk c} w_s x_s[p] B_s[n],   w_s = dt_s exp(acs_last - acs_s)
+//   S_k[p][n] = sum_{s in block k} w_s x_s[p] B_s[n],   w_s = dt_s exp(acs_last - acs_s)
 //
-// computed transposed as one M=128 (n) x N=64 (p) x K=256 (s) product per (batch, chunk,
-// head): A = B_c^T and the B operand X'' = diag(w) x_c, both read MN-major straight from the
-// 128-byte-swizzled tiles that TMA writes.  The fp32 chunk state feeds the float32 state
-// pass and finally h_final, whose tolerance (1e-3 relative to its RMS) is tighter than one
-// bf16 rounding of w_s x_s (RMS relative error 2^-9/sqrt(3) = 1.1e-3).  So X'' is split
+// for every 128-token block k (the M of one tcgen05 MMA; the tensor-core path blocks the
+// sequence in 128 tokens whatever chunk the caller asked for -- the decomposition is exact,
+// only rounding differs), computed transposed as one M=128 (n) x N=64 (p) x K=128 (s)
+// product per (batch, block, head): A = B_k^T and the B operand X'' = diag(w) x_k, both read
+// MN-major straight from 128-byte-swizzled tiles.  The fp32 block state feeds the float32
+// state pass and finally h_final, whose tolerance (1e-3 relative to its RMS) is tighter than
+// one bf16 rounding of w_s x_s (RMS relative error 2^-9/sqrt(3) = 1.1e-3).  So X'' is split
 // into bf16 hi + lo parts (hi = bf16(v), lo = bf16(v - hi), |v - hi - lo| <= 2^-17 |v|) and
-// both are accumulated into the same fp32 TMEM accumulator: 2 x 16 MMAs of K=16.
+// both are accumulated into the same fp32 TMEM accumulator: 2 x 8 MMAs of K=16.
 //
-// Source: the chunk state that the blog walk-through of "Compiler-First State Space
+// Source: the per-chunk state that the blog walk-through of "Compiler-First State Space
 // Duality and Portable O(1) Autoregressive Caching for Inference" (bqwf.cn) §1.1 says is
 // passed between chunks (the decay-weighted B^T X of each chunk).
 //
-// Structure: persistent CTAs (one per SM, 128 threads); CTA k owns a contiguous range of
-// (batch, chunk, head) items, so consecutive items share the chunk's B tile (64 KB, loaded
-// once per (batch, chunk, group)).  Per item: TMA the x tile [256 x 64] bf16 and bulk-copy
-// the item's dt and cumsum rows into one of two stages (the next item's data loads while
-// this one computes, so no global load sits on the critical path), scale rows by w_s into hi
-// (in place) and lo, one thread issues the 32 MMAs into one of two TMEM accumulators, and
-// the previous item's accumulator is drained to global memory meanwhile.
+// Structure: persistent CTAs, one per SM, each owning a contiguous range of (batch, block,
+// head) items (consecutive items share the block's B tile).  Warp-specialised:
+//   warp 0      TMA producer: B tile per (batch, block, group); x tile + the item's
+//               per-token factors into a ring of kStages stages
+//   warp 1      MMA issuer (one lane): 16 MMAs per item into one of two TMEM accumulators
+//   warps 2..9  workers: scale rows by w into hi (in place) and lo; drain the accumulator of
+//               the item before to global memory
+// The roles meet only at mbarriers (full/empty per stage, per accumulator, per B tile), so
+// the tensor core runs back to back while the workers transform and drain other items.
 #include "common.cuh"
 #include "launch.h"
 #include "tc.cuh"
@@ -30,244 +33,256 @@
 namespace ssd {
 
 namespace cst {
-constexpr int Q = 256, P = 64, N = 128;
-constexpr int kThreads = 256;  // 8 warps: two per TMEM lane quarter
-constexpr uint32_t kTileX = Q * P * 2;  // 32 KB
-constexpr uint32_t kTileB = Q * N * 2;  // 64 KB (two 64-wide n halves)
-constexpr uint32_t kOffB = 0;
-constexpr uint32_t kOffX0 = kOffB + kTileB;
-constexpr uint32_t kOffLo0 = kOffX0 + kTileX;
-constexpr uint32_t kOffX1 = kOffLo0 + kTileX;
-constexpr uint32_t kOffLo1 = kOffX1 + kTileX;
-constexpr uint32_t kOffW = kOffLo1 + kTileX;          // w_s, 2 x 256 floats
-constexpr uint32_t kOffRows = kOffW + 2 * Q * 4;      // per stage: dt[256], acs[256]
-constexpr uint32_t kRowBytes = 2 * Q * 4;
-constexpr uint32_t kOffBar = kOffRows + 2 * kRowBytes;
-constexpr uint32_t kSmem = kOffBar + 64 + 1024;  // + slack for 1024-byte alignment
+constexpr int R = 128, P = 64, N = 128;
+constexpr int kWorkers = 8;
+constexpr int kThreads = (2 + kWorkers) * 32;
+constexpr int kStages = 4;
+constexpr uint32_t kBox = R * 128;                 // [128 rows][64 bf16], 16 KB
+constexpr uint32_t kOffB = 0;                      // B block: 2 n-boxes, 32 KB
+constexpr uint32_t kStageBytes = 2 * kBox + 1024;  // x/hi box, lo box, colv[128] + acs2[128]
+constexpr uint32_t kOffStage = 2 * kBox;
+constexpr uint32_t kOffBar = kOffStage + kStages * kStageBytes;
+constexpr uint32_t kSmem = kOffBar + 256 + 1024;  // + slack for 1024-byte alignment
 constexpr uint32_t kTmemCols = 128;               // two 64-column fp32 accumulators
 }  // namespace cst
 
 __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
     const float *__restrict__ dtf, const float *__restrict__ acs, float *__restrict__ states,
-    int *__restrict__ status, int H, int G, int nc, int total) {
+    int *__restrict__ status, int H, int G, int nk, int total) {
     using namespace cst;
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bar_b = reinterpret_cast<uint64_t *>(smem + kOffBar);
-    uint64_t *bar_x = bar_b + 1;    // [2]
-    uint64_t *bar_mma = bar_b + 3;  // [2]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_b + 5);
-    float *wbuf = reinterpret_cast<float *>(smem + kOffW);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    uint64_t *st_full = bars;                 // [kStages] TMA -> workers
+    uint64_t *op_full = st_full + kStages;    // [kStages] workers -> MMA (operands written)
+    uint64_t *st_empty = op_full + kStages;   // [kStages] MMA commit -> producer
+    uint64_t *acc_full = st_empty + kStages;  // [2] MMA commit -> workers
+    uint64_t *acc_empty = acc_full + 2;       // [2] workers -> MMA
+    uint64_t *b_full = acc_empty + 2;         // B tile landed
+    uint64_t *b_empty = b_full + 1;           // MMA commit after the last item of a tile
+    uint64_t *fin = b_empty + 1;              // MMA commit after the last MMA of the CTA
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int first = (int)((long long)blockIdx.x * total / gridDim.x);
     const int cnt = (int)((long long)(blockIdx.x + 1) * total / gridDim.x) - first;
     if (cnt <= 0) return;
     const int hpg = H / G;
-    const size_t Lp = (size_t)nc * Q;
+    const size_t Lp = (size_t)nk * R;
 
     if (tid == 0) {
-        mbar_init(bar_b, 1);
-        mbar_init(&bar_x[0], 1);
-        mbar_init(&bar_x[1], 1);
-        mbar_init(&bar_mma[0], 1);
-        mbar_init(&bar_mma[1], 1);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&st_full[i], 1);
+            mbar_init(&op_full[i], kWorkers);
+            mbar_init(&st_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], kWorkers);
+        }
+        mbar_init(b_full, 1);
+        mbar_init(b_empty, 1);
+        mbar_init(fin, 1);
+        *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tm_x);
         tma_prefetch_desc(&tm_b);
     }
-    if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+    if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // item -> (b, c, h); the B tile depends on (b, c, g)
-    auto item_bch = [&](int j, int &b, int &c, int &h) {
+    auto item = [&](int j, int &b, int &k, int &h) {
         const int it = first + j;
         h = it % H;
         const int t = it / H;
-        c = t % nc;
-        b = t / nc;
+        k = t % nk;
+        b = t / nk;
     };
     auto b_key = [&](int j) {
-        int b, c, h;
-        item_bch(j, b, c, h);
-        return (b * nc + c) * G + h / hpg;
+        int b, k, h;
+        item(j, b, k, h);
+        return (b * nk + k) * G + h / hpg;
     };
-    auto issue_x = [&](int j) {  // thread 0 only: x tile plus the item's dt and acs rows
-        int b, c, h;
-        item_bch(j, b, c, h);
-        const int s = j & 1;
-        const size_t row = ((size_t)b * H + h) * Lp + (size_t)c * Q;
-        uint8_t *rows = smem + kOffRows + s * kRowBytes;
-        mbar_arrive_expect_tx(&bar_x[s], kTileX + kRowBytes);
-        tma_load_3d(smem + (s ? kOffX1 : kOffX0), &tm_x, h * P, c * Q, b, &bar_x[s]);
-        bulk_load(rows, dtf + row, Q * 4, &bar_x[s]);
-        bulk_load(rows + Q * 4, acs + row, Q * 4, &bar_x[s]);
-    };
-    auto issue_b = [&](int j) {  // thread 0 only
-        int b, c, h;
-        item_bch(j, b, c, h);
-        const int g = h / hpg;
-        mbar_arrive_expect_tx(bar_b, kTileB);
-        tma_load_3d(smem + kOffB, &tm_b, g * N, c * Q, b, bar_b);
-        tma_load_3d(smem + kOffB + kTileB / 2, &tm_b, g * N + 64, c * Q, b, bar_b);
-    };
-
-    // bookkeeping of outstanding asynchronous operations, identical in every thread
-    int x_issued[2] = {0, 0}, x_done[2] = {0, 0};
-    int b_issued = 0, b_done = 0;
-    int mma_issued[2] = {0, 0}, mma_done[2] = {0, 0};
-    bool ok = true;
-
-    auto epilogue = [&](int j) {
-        const int s = j & 1;
-        ok = mbar_wait_all(&bar_mma[s], mma_done[s] & 1, status);
-        if (!ok) return;
-        ++mma_done[s];
-        tc_fence_after();
-        int b, c, h;
-        item_bch(j, b, c, h);
-        float *out = states + (((size_t)b * nc + c) * H + h) * (size_t)(P * N);
-        // warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 and split the 64 columns
-        const int quarter = warp & 3, colhalf = warp >> 2;
-        const int n = quarter * 32 + lane;
-        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * 64 + colhalf * 32);
-        float v0[16], v1[16];
-        tmem_ld16(taddr, v0);
-        tmem_ld16(taddr + 16, v1);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) out[(size_t)(colhalf * 32 + i) * N + n] = v0[i];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) out[(size_t)(colhalf * 32 + 16 + i) * N + n] = v1[i];
-        tc_fence_before();
-    };
-
-    if (tid == 0) {
-        issue_b(0);
-        issue_x(0);
-    }
-    b_issued = 1;
-    x_issued[0] = 1;
-
-    for (int j = 0; j < cnt && ok; ++j) {
-        const int s = j & 1;
-        // prefetch the next item's x tile into the other stage once MMA j-1 has read it
-        if (j + 1 < cnt) {
-            if (j >= 1) ok = mbar_wait_all(&bar_mma[s ^ 1], mma_done[s ^ 1] & 1, status);
-            if (!ok) break;
-            if (tid == 0) issue_x(j + 1);
-            ++x_issued[s ^ 1];
-        }
-        // B tile of this item (reloaded when (batch, chunk, group) changes)
-        if (j > 0 && b_key(j) != b_key(j - 1)) {
-            ok = mbar_wait_all(&bar_mma[s ^ 1], mma_done[s ^ 1] & 1, status);  // MMA j-1 done
-            if (!ok) break;
-            if (tid == 0) issue_b(j);
-            ++b_issued;
-        }
-        if (b_done < b_issued) {
-            ok = mbar_wait_all(bar_b, b_done & 1, status);
-            if (!ok) break;
-            ++b_done;
-        }
-        ok = mbar_wait_all(&bar_x[s], x_done[s] & 1, status);
-        if (!ok) break;
-        ++x_done[s];
-
-        // row weights w_s = dt_s exp(acs_last - acs_s) (0 past the end of the sequence)
-        const float *dt_row = reinterpret_cast<const float *>(smem + kOffRows + s * kRowBytes);
-        const float *acs_row = dt_row + Q;
-        const float a_last = acs_row[Q - 1];
-        for (int r = tid; r < Q; r += kThreads) wbuf[s * Q + r] = dt_row[r] * expf(a_last - acs_row[r]);
-        __syncthreads();
-
-        // x -> hi (in place) and lo, same swizzled positions
-        uint8_t *xt = smem + (s ? kOffX1 : kOffX0);
-        uint8_t *lo = smem + (s ? kOffLo1 : kOffLo0);
-#pragma unroll 4
-        for (int q = tid; q < Q * 8; q += kThreads) {
-            const int row = q >> 3, chunk = q & 7;
-            const uint32_t off = sw128_offset(row, chunk);
-            uint4 raw = *reinterpret_cast<const uint4 *>(xt + off);
-            const float w = wbuf[s * Q + row];
-            uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
-            uint32_t hi[4], lw[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                __nv_bfloat162 v2 = *reinterpret_cast<__nv_bfloat162 *>(&in[i]);
-                const float2 f = __bfloat1622float2(v2);
-                const float a0 = f.x * w, a1 = f.y * w;
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(a0, a1);
-                const float2 hf = __bfloat1622float2(h2);
-                const __nv_bfloat162 l2 = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
-                hi[i] = *reinterpret_cast<const uint32_t *>(&h2);
-                lw[i] = *reinterpret_cast<const uint32_t *>(&l2);
+    auto new_tile = [&](int j) { return j == 0 || b_key(j) != b_key(j - 1); };
+    auto last_of_tile = [&](int j) { return j == cnt - 1 || b_key(j + 1) != b_key(j); };
+    auto stage = [&](int j) { return smem + kOffStage + (uint32_t)(j % kStages) * kStageBytes; };
+    // a bounded wait that gives up at once when another role has already timed out
+    auto wait = [&](uint64_t *bar, uint32_t parity) {
+        while (!mbar_test(bar, parity)) {
+            if (*abort_flag) return false;
+            if (!mbar_wait(bar, parity, status)) {
+                *abort_flag = 1;
+                return false;
             }
-            *reinterpret_cast<uint4 *>(xt + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4 *>(lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            return true;
         }
-        fence_proxy_async_smem();
-        __syncthreads();
+        return true;
+    };
 
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t d = tmem + (uint32_t)(s * 64);
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            int tiles = 0;
+            for (int j = 0; j < cnt; ++j) {
+                int b, k, h;
+                item(j, b, k, h);
+                if (new_tile(j)) {
+                    if (tiles > 0 && !wait(b_empty, (tiles - 1) & 1)) break;
+                    mbar_arrive_expect_tx(b_full, 2 * kBox);
+                    const int g = h / hpg;
+                    tma_load_3d(smem + kOffB, &tm_b, g * N, k * R, b, b_full);
+                    tma_load_3d(smem + kOffB + kBox, &tm_b, g * N + 64, k * R, b, b_full);
+                    ++tiles;
+                }
+                const int s = j % kStages;
+                if (j >= kStages && !wait(&st_empty[s], ((j / kStages) - 1) & 1)) break;
+                uint8_t *st = stage(j);
+                const size_t row = ((size_t)b * H + h) * Lp + (size_t)k * R;
+                mbar_arrive_expect_tx(&st_full[s], kBox + 2 * R * 4);
+                tma_load_3d(st, &tm_x, h * P, k * R, b, &st_full[s]);
+                bulk_load(st + 2 * kBox, dtf + row, R * 4, &st_full[s]);
+                bulk_load(st + 2 * kBox + R * 4, acs + row, R * 4, &st_full[s]);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(128, 64, true, true);
             const uint32_t a0 = smem_u32(smem + kOffB);
-            const uint32_t bh = smem_u32(xt), bl = smem_u32(lo);
+            int tiles = 0;
+            for (int j = 0; j < cnt; ++j) {
+                const int s = j % kStages, a = j & 1;
+                if (new_tile(j)) {
+                    if (!wait(b_full, tiles & 1)) break;
+                    ++tiles;
+                }
+                if (!wait(&op_full[s], (j / kStages) & 1)) break;
+                if (j >= 2 && !wait(&acc_empty[a], ((j >> 1) - 1) & 1)) break;
+                tc_fence_after();
+                uint8_t *st = stage(j);
+                const uint32_t bh = smem_u32(st), bl = smem_u32(st + kBox);
+                const uint32_t d = tmem + (uint32_t)(a * 64);
 #pragma unroll 1
-            for (int k = 0; k < Q / 16; ++k)
-                mma_ss(d, desc_mnmajor_sw128(a0 + k * 2048, kTileB / 2), desc_mnmajor_sw128(bh + k * 2048, kTileX),
-                       idesc, k > 0 ? 1u : 0u);
+                for (int kk = 0; kk < R / 16; ++kk)
+                    mma_ss(d, desc_mnmajor_sw128(a0 + kk * 2048, kBox), desc_mnmajor_sw128(bh + kk * 2048, kBox),
+                           idesc, kk > 0 ? 1u : 0u);
 #pragma unroll 1
-            for (int k = 0; k < Q / 16; ++k)
-                mma_ss(d, desc_mnmajor_sw128(a0 + k * 2048, kTileB / 2), desc_mnmajor_sw128(bl + k * 2048, kTileX),
-                       idesc, 1u);
-            mma_commit(&bar_mma[s]);
+                for (int kk = 0; kk < R / 16; ++kk)
+                    mma_ss(d, desc_mnmajor_sw128(a0 + kk * 2048, kBox), desc_mnmajor_sw128(bl + kk * 2048, kBox),
+                           idesc, 1u);
+                mma_commit(&acc_full[a]);
+                mma_commit(&st_empty[s]);
+                if (last_of_tile(j)) mma_commit(b_empty);
+            }
+            // every MMA (and every arrive it triggers) has landed before TMEM is released
+            mma_commit(fin);
+            mbar_wait(fin, 0, status);
         }
-        ++mma_issued[s];
-        if (j >= 1) epilogue(j - 1);
+    } else {
+        // ---------------------------------------------------------------- workers
+        const int wk = warp - 2;  // 0..7: rows [16 wk, 16 wk + 16) of the transform
+        const int quarter = warp & 3, colhalf = wk >> 2;  // epilogue: TMEM lane quarter, column half
+        auto epilogue = [&](int j) {
+            const int a = j & 1;
+            if (!wait(&acc_full[a], (j >> 1) & 1)) return false;
+            tc_fence_after();
+            int b, k, h;
+            item(j, b, k, h);
+            float *out = states + (((size_t)b * nk + k) * H + h) * (size_t)(P * N);
+            const int n = quarter * 32 + lane;
+            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 64 + colhalf * 32);
+            float v0[16], v1[16];
+            tmem_ld16(taddr, v0);
+            tmem_ld16(taddr + 16, v1);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[a]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) out[(size_t)(colhalf * 32 + i) * N + n] = v0[i];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) out[(size_t)(colhalf * 32 + 16 + i) * N + n] = v1[i];
+            return true;
+        };
+        for (int j = 0; j < cnt; ++j) {
+            const int s = j % kStages;
+            if (!wait(&st_full[s], (j / kStages) & 1)) break;
+            uint8_t *xt = stage(j);
+            uint8_t *lo = xt + kBox;
+            const float *colv = reinterpret_cast<const float *>(xt + 2 * kBox);
+            const float *acs2 = colv + R;
+            // w_s = dt_s exp(acs_last - acs_s) = exp2(acs2_last - colv_s); lanes 0..15 hold the
+            // weights of this warp's 16 rows
+            const float wl = lane < 16 ? ex2_approx(acs2[R - 1] - colv[wk * 16 + lane]) : 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {  // 16 rows x 8 chunks = 128 chunks over 32 lanes
+                const int idx = q * 32 + lane;
+                const int rl = idx >> 3, chunk = idx & 7;
+                const int row = wk * 16 + rl;
+                const float w = __shfl_sync(0xffffffffu, wl, rl);
+                const uint32_t off = sw128_offset(row, chunk);
+                uint4 raw = *reinterpret_cast<const uint4 *>(xt + off);
+                uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
+                uint32_t hi[4], lw[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&in[i]));
+                    const float a0 = f.x * w, a1 = f.y * w;
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(a0, a1);
+                    const float2 hf = __bfloat1622float2(h2);
+                    const __nv_bfloat162 l2 = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
+                    hi[i] = *reinterpret_cast<const uint32_t *>(&h2);
+                    lw[i] = *reinterpret_cast<const uint32_t *>(&l2);
+                }
+                *reinterpret_cast<uint4 *>(xt + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&op_full[s]);
+            if (j >= 1 && !epilogue(j - 1)) break;
+        }
+        if (!*abort_flag) epilogue(cnt - 1);
     }
-    if (ok) epilogue(cnt - 1);
 
-    if (!ok) {
-        // a wait timed out: drain what is still in flight (bounded) before releasing TMEM
-        for (int s = 0; s < 2; ++s) {
-            while (mma_done[s] < mma_issued[s] && mbar_wait(&bar_mma[s], mma_done[s] & 1, nullptr)) ++mma_done[s];
-            while (x_done[s] < x_issued[s] && mbar_wait(&bar_x[s], x_done[s] & 1, nullptr)) ++x_done[s];
+    __syncthreads();
+    if (*abort_flag && tid == 0) {
+        // a wait timed out: let copies still in flight land (bounded) before the CTA exits
+        const unsigned long long t0 = globaltimer();
+        while (globaltimer() - t0 < 2000000ull) {
         }
-        while (b_done < b_issued && mbar_wait(bar_b, b_done & 1, nullptr)) ++b_done;
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_free(tmem, kTmemCols);
+    if (warp == 1) tmem_free(tmem, kTmemCols);
 }
 
-bool chunk_state_tc_supported(int dtype, int P, int N, int chunk) {
-    return dtype == SSD_DTYPE_BF16 && P == cst::P && N == cst::N && chunk == cst::Q;
+bool prefill_tc_supported(int dtype, int P, int N) {
+    return dtype == SSD_DTYPE_BF16 && P == cst::P && N == cst::N;
 }
 
 cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const float *dtf, const float *acs,
                                   float *states, int *status, int B, int L, int H, int G,
                                   int num_sms, cudaStream_t st) {
     using namespace cst;
-    const int nc = cdiv(L, Q);
-    const int total = B * nc * H;
+    const int nk = cdiv(L, R);
+    const int total = B * nk * H;
     CUtensorMap tm_x, tm_b;
     cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B,
-                                      (uint64_t)H * P * 2, (uint64_t)L * H * P * 2, 64, Q, 1);
+                                      (uint64_t)H * P * 2, (uint64_t)L * H * P * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
     e = make_tmap_bf16_3d(&tm_b, Bm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)G * N * 2,
-                          (uint64_t)L * G * N * 2, 64, Q, 1);
+                          (uint64_t)L * G * N * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
     const int grid = total < num_sms ? total : num_sms;
     cudaFuncSetAttribute(chunk_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
-    chunk_state_tc_kernel<<<grid, kThreads, kSmem, st>>>(tm_x, tm_b, dtf, acs, states, status, H, G, nc,
+    chunk_state_tc_kernel<<<grid, kThreads, kSmem, st>>>(tm_x, tm_b, dtf, acs, states, status, H, G, nk,
                                                          total);
     return cudaGetLastError();
 }

@@ -1,6 +1,7 @@
 // launch.h -- internal launchers of the SSD kernels (not part of the public C ABI).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 
@@ -8,35 +9,45 @@ namespace ssd {
 
 // Prefill workspace layout, 256-byte aligned pieces:
 //   status int32 (256-byte slot): SSD_OK, or SSD_ERR_TIMEOUT if a bounded wait gave up
-//   dtf    [B][H][Lp]          clipped dt per token (0 past the end of the sequence)
-//   acs    [B][H][Lp]          inclusive cumsum of dt*A inside each chunk
-//   states [B][nc][H][P][N]    chunk states, overwritten in place by the state each
-//                              chunk starts from (h_prev)
-// with nc = ceil(L / chunk), Lp = nc * chunk.
+//   dtf    [B][H][Lp]          clipped dt per token (0 past the end of the sequence); on the
+//                              tensor-core path colv = acs2 - log2(dt) instead
+//   acs    [B][H][Lp]          inclusive cumsum of dt*A inside each block; on the tensor-core
+//                              path acs2 = that cumsum times log2(e)
+//   states [B][nb][H][P][N]    fp32 block states; the CUDA-core path overwrites them in
+//                              place with the state each block starts from (h_prev)
+//   hT     [B][nb][H][N][P]    (tensor-core path) h_prev of each block, bf16, transposed
+// with nb = ceil(L / block), Lp = nb * block.  The block is the caller's chunk on the
+// CUDA-core path and 128 tokens (the tcgen05 M) on the tensor-core path.
 struct PrefillWorkspace {
     int *status;
     float *dtf;
     float *acs;
     float *states;
+    __nv_bfloat16 *hT;
 };
-size_t prefill_workspace_bytes(int B, int L, int H, int P, int N, int chunk);
-PrefillWorkspace carve_prefill_workspace(void *base, int B, int L, int H, int P, int N, int chunk);
+size_t prefill_workspace_bytes(int B, int L, int H, int P, int N, int block, bool transposed_bf16);
+PrefillWorkspace carve_prefill_workspace(void *base, int B, int L, int H, int P, int N, int block,
+                                         bool transposed_bf16);
 
+// log2_form: write colv = acs*log2(e) - log2(dt) and acs2 = acs*log2(e) (tensor-core path)
+// instead of dt and acs.
 cudaError_t launch_decay_prep(int dtype, const void *dt, const float *A_log, const float *dt_bias,
                               float dt_min, float dt_max, float *dtf, float *acs, int *status, int B,
-                              int L, int H, int chunk, cudaStream_t st);
+                              int L, int H, int chunk, bool log2_form, cudaStream_t st);
 
-// tensor-core chunk state (bf16 storage, P = 64, N = 128, chunk 256)
-bool chunk_state_tc_supported(int dtype, int P, int N, int chunk);
+// tensor-core prefill (bf16 storage, P = 64, N = 128), 128-token blocks
+constexpr int kTcBlock = 128;
+bool prefill_tc_supported(int dtype, int P, int N);
 cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const float *dtf, const float *acs,
                                   float *states, int *status, int B, int L, int H, int G,
                                   int num_sms, cudaStream_t st);
 
-// tensor-core chunk scan (bf16 storage, P = 64, N = 128, chunk 256)
-bool chunk_scan_tc_supported(int dtype, int P, int N, int chunk);
 cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, const float *dtf,
-                                 const float *acs, const float *hprev, const float *D, void *y,
+                                 const float *acs, const __nv_bfloat16 *hT, const float *D, void *y,
                                  int *status, int B, int L, int H, int G, int num_sms, cudaStream_t st);
+cudaError_t launch_state_pass_t(const float *states, const float *acs, const float *h0, float *h_final,
+                                __nv_bfloat16 *hT, int B, int L, int H, int P, int N, int chunk,
+                                cudaStream_t st);
 
 cudaError_t launch_chunk_state(int dtype, const void *x, const void *Bm, const float *dtf,
                                const float *acs, float *states, int B, int L, int H, int G, int N,

@@ -41,11 +41,22 @@ def test_status_strings_and_version():
     assert L.ssd_last_cuda_error() == 0
 
 
-def ws_bytes(B, Lx, H, P, N, chunk):
-    nc = -(-Lx // chunk)
-    per_tok = -(-4 * B * H * nc * chunk // 256) * 256
-    states = -(-4 * B * nc * H * P * N // 256) * 256
-    return 256 + 2 * per_tok + states
+def _layout(B, Lx, H, P, N, block, transposed):
+    up = lambda v: -(-v // 256) * 256
+    nb = -(-Lx // block)
+    per_tok = up(4 * B * H * nb * block)
+    states = up(4 * B * nb * H * P * N)
+    hT = up(2 * B * nb * H * P * N) if transposed else 0
+    return 256 + 2 * per_tok + states + hT
+
+
+def ws_bytes(B, Lx, H, P, N, chunk, tensor_core_shape):
+    """The larger of the CUDA-core layout (caller's chunk) and, for bf16 P=64 N=128, the
+    tensor-core layout (128-token blocks plus a bf16 copy of the carried states)."""
+    need = _layout(B, Lx, H, P, N, chunk, False)
+    if tensor_core_shape:
+        need = max(need, _layout(B, Lx, H, P, N, 128, True))
+    return need
 
 
 @pytest.mark.parametrize("shape", [(1, 4096, 80, 64, 1, 128, 256), (8, 2048, 64, 64, 1, 128, 256),
@@ -54,7 +65,9 @@ def ws_bytes(B, Lx, H, P, N, chunk):
 def test_prefill_workspace_size(shape):
     B, Lx, H, P, G, N, chunk = shape
     got = L.ssd_chunk_scan_workspace_size(B, Lx, H, P, G, N, chunk, BF16)
-    assert got == ws_bytes(B, Lx, H, P, N, chunk) and got % 256 == 0
+    assert got == ws_bytes(B, Lx, H, P, N, chunk, P == 64 and N == 128) and got % 256 == 0
+    got32 = L.ssd_chunk_scan_workspace_size(B, Lx, H, P, G, N, chunk, F32)
+    assert got32 == ws_bytes(B, Lx, H, P, N, chunk, False)
     assert L.ssd_chunk_scan_workspace_size(0, Lx, H, P, G, N, chunk, BF16) == 0
     assert L.ssd_chunk_scan_workspace_size(B, Lx, H, 32, G, N, chunk, BF16) == 0   # unsupported P
 
