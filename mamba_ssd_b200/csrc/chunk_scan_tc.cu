@@ -27,7 +27,7 @@
 //   warp 0      TMA producer: C/B tiles per (batch, block, group); x tile, h_prev^T tile and
 //               the item's per-token factors into a ring of kStages stages
 //   warp 1      MMA issuer (one lane): CB per tile; O and Y per item into one of two TMEM sets
-//   warps 2..9  workers: P~ of item j into TMEM, then the epilogue of item j - 1
+//   warps 2..17 workers: P~ of item j into TMEM, then the epilogue of item j - 1
 // so the tensor core runs item j's products while the CUDA cores form item j+1's P~ and
 // write item j-1's outputs.
 #include "common.cuh"
@@ -39,7 +39,7 @@ namespace ssd {
 
 namespace csc {
 constexpr int R = 128, P = 64, N = 128;
-constexpr int kWorkers = 8;
+constexpr int kWorkers = 16;
 constexpr int kThreads = (2 + kWorkers) * 32;
 constexpr int kStages = 4;
 constexpr uint32_t kBox = R * 128;            // [128 rows][64 bf16] swizzled box: 16 KB
@@ -214,9 +214,9 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
         }
     } else {
         // ---------------------------------------------------------------- workers
-        // warps w, w + 4 share TMEM lanes 32 (w % 4) .. + 31 (rows of the block); the two
-        // halves split P~'s column blocks and the output columns
-        const int rq = warp & 3, ch = (warp - 2) >> 2;
+        // warps w, w + 4, w + 8, w + 12 share TMEM lanes 32 (w % 4) .. + 31 (rows of the
+        // block); the four split P~'s 32-column blocks and the 16-column output quarters
+        const int rq = warp & 3, cq = (warp - 2) >> 2;
         const int myrow = rq * 32 + lane;
         const uint32_t lane_base = (uint32_t)(rq * 32) << 16;
         auto epilogue = [&](int j, float scale) {
@@ -226,20 +226,18 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
             int b, k, h;
             item(j, b, k, h);
             const uint32_t set = tmem + lane_base + kSet0 + t * kSet;
-            float yv[32], ov[32];
-            tmem_ld16(set + kOffY + ch * 32, *reinterpret_cast<float(*)[16]>(&yv[0]));
-            tmem_ld16(set + kOffY + ch * 32 + 16, *reinterpret_cast<float(*)[16]>(&yv[16]));
-            tmem_ld16(set + kOffO + ch * 32, *reinterpret_cast<float(*)[16]>(&ov[0]));
-            tmem_ld16(set + kOffO + ch * 32 + 16, *reinterpret_cast<float(*)[16]>(&ov[16]));
+            float yv[16], ov[16];
+            tmem_ld16(set + kOffY + cq * 16, yv);
+            tmem_ld16(set + kOffO + cq * 16, ov);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[t]);
             const int tok = k * R + myrow;
             if (tok < L) {
-                uint4 *yr = reinterpret_cast<uint4 *>(y + (((size_t)b * L + tok) * H + h) * P + ch * 32);
+                uint4 *yr = reinterpret_cast<uint4 *>(y + (((size_t)b * L + tok) * H + h) * P + cq * 16);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 2; ++q) {
                     uint32_t o[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
@@ -270,8 +268,8 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
             const float al = acs2[myrow];
             const float d = D ? __ldg(D + h) : 0.f;
             const uint32_t set = tmem + kSet0 + t * kSet;
-#pragma unroll 1
-            for (int blk = ch; blk < 4; blk += 2) {
+            {
+                const int blk = cq;  // one 32-column block of P~ per warp
                 uint32_t packed[16];
                 if (blk > rq) {  // entirely above the diagonal for these rows
 #pragma unroll
@@ -282,22 +280,21 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
                     tmem_ld16(tmem + lane_base + kColCB + blk * 32 + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
                     tmem_wait_ld();
                     const float4 *c4 = reinterpret_cast<const float4 *>(colv + blk * 32);
-                    float pr[32];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const float4 c = c4[i];
-                        pr[4 * i + 0] = v[4 * i + 0] * ex2_approx(al - c.x);
-                        pr[4 * i + 1] = v[4 * i + 1] * ex2_approx(al - c.y);
-                        pr[4 * i + 2] = v[4 * i + 2] * ex2_approx(al - c.z);
-                        pr[4 * i + 3] = v[4 * i + 3] * ex2_approx(al - c.w);
+                        v[4 * i + 0] *= ex2_approx(al - c.x);
+                        v[4 * i + 1] *= ex2_approx(al - c.y);
+                        v[4 * i + 2] *= ex2_approx(al - c.z);
+                        v[4 * i + 3] *= ex2_approx(al - c.w);
                     }
                     if (blk == rq) {  // the diagonal block: causal mask and the D skip
                         const int ld = myrow - blk * 32;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) pr[i] = i < ld ? pr[i] : (i == ld ? pr[i] + d : 0.f);
+                        for (int i = 0; i < 32; ++i) v[i] = i < ld ? v[i] : (i == ld ? v[i] + d : 0.f);
                     }
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(pr[2 * i], pr[2 * i + 1]);
+                    for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
                 }
                 tmem_st16(set + lane_base + kOffPT + blk * 16, packed);
             }

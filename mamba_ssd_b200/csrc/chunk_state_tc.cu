@@ -2,6 +2,8 @@
 //
 //   S_k[p][n] = sum_{s in block k} w_s x_s[p] B_s[n],   w_s = dt_s exp(acs_last - acs_s)
 //
+// stored transposed as S_k^T [N][P] (the layout of the accumulator: TMEM lane n, column p)
+//
 // for every 128-token block k (the M of one tcgen05 MMA; the tensor-core path blocks the
 // sequence in 128 tokens whatever chunk the caller asked for -- the decomposition is exact,
 // only rounding differs), computed transposed as one M=128 (n) x N=64 (p) x K=128 (s)
@@ -21,8 +23,8 @@
 //   warp 0      TMA producer: B tile per (batch, block, group); x tile + the item's
 //               per-token factors into a ring of kStages stages
 //   warp 1      MMA issuer (one lane): 16 MMAs per item into one of two TMEM accumulators
-//   warps 2..9  workers: scale rows by w into hi (in place) and lo; drain the accumulator of
-//               the item before to global memory
+//   warps 2..17 workers: scale rows by w into hi (in place) and lo; drain the accumulator of
+//               the item before to global memory (the state is written transposed, [N][P])
 // The roles meet only at mbarriers (full/empty per stage, per accumulator, per B tile), so
 // the tensor core runs back to back while the workers transform and drain other items.
 #include "common.cuh"
@@ -34,7 +36,7 @@ namespace ssd {
 
 namespace cst {
 constexpr int R = 128, P = 64, N = 128;
-constexpr int kWorkers = 8;
+constexpr int kWorkers = 16;
 constexpr int kThreads = (2 + kWorkers) * 32;
 constexpr int kStages = 4;
 constexpr uint32_t kBox = R * 128;                 // [128 rows][64 bf16], 16 KB
@@ -186,28 +188,27 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
         }
     } else {
         // ---------------------------------------------------------------- workers
-        const int wk = warp - 2;  // 0..7: rows [16 wk, 16 wk + 16) of the transform
-        const int quarter = warp & 3, colhalf = wk >> 2;  // epilogue: TMEM lane quarter, column half
+        const int wk = warp - 2;  // 0..15: rows [8 wk, 8 wk + 8) of the transform
+        const int quarter = warp & 3, colq = wk >> 2;  // epilogue: TMEM lane quarter, column quarter
         auto epilogue = [&](int j) {
             const int a = j & 1;
             if (!wait(&acc_full[a], (j >> 1) & 1)) return false;
             tc_fence_after();
             int b, k, h;
             item(j, b, k, h);
-            float *out = states + (((size_t)b * nk + k) * H + h) * (size_t)(P * N);
-            const int n = quarter * 32 + lane;
-            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 64 + colhalf * 32);
-            float v0[16], v1[16];
+            // S^T[n][p] row n = this lane, 16 columns: 64 contiguous bytes
+            float *out = states + (((size_t)b * nk + k) * H + h) * (size_t)(P * N) +
+                         (size_t)(quarter * 32 + lane) * P + colq * 16;
+            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 64 + colq * 16);
+            float v0[16];
             tmem_ld16(taddr, v0);
-            tmem_ld16(taddr + 16, v1);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[a]);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) out[(size_t)(colhalf * 32 + i) * N + n] = v0[i];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) out[(size_t)(colhalf * 32 + 16 + i) * N + n] = v1[i];
+            for (int q = 0; q < 4; ++q)
+                reinterpret_cast<float4 *>(out)[q] = make_float4(v0[4 * q], v0[4 * q + 1], v0[4 * q + 2], v0[4 * q + 3]);
             return true;
         };
         for (int j = 0; j < cnt; ++j) {
@@ -217,14 +218,14 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
             uint8_t *lo = xt + kBox;
             const float *colv = reinterpret_cast<const float *>(xt + 2 * kBox);
             const float *acs2 = colv + R;
-            // w_s = dt_s exp(acs_last - acs_s) = exp2(acs2_last - colv_s); lanes 0..15 hold the
-            // weights of this warp's 16 rows
-            const float wl = lane < 16 ? ex2_approx(acs2[R - 1] - colv[wk * 16 + lane]) : 0.f;
+            // w_s = dt_s exp(acs_last - acs_s) = exp2(acs2_last - colv_s); lanes 0..7 hold the
+            // weights of this warp's 8 rows
+            const float wl = lane < 8 ? ex2_approx(acs2[R - 1] - colv[wk * 8 + lane]) : 0.f;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {  // 16 rows x 8 chunks = 128 chunks over 32 lanes
+            for (int q = 0; q < 2; ++q) {  // 8 rows x 8 chunks = 64 chunks over 32 lanes
                 const int idx = q * 32 + lane;
                 const int rl = idx >> 3, chunk = idx & 7;
-                const int row = wk * 16 + rl;
+                const int row = wk * 8 + rl;
                 const float w = __shfl_sync(0xffffffffu, wl, rl);
                 const uint32_t off = sw128_offset(row, chunk);
                 uint4 raw = *reinterpret_cast<const uint4 *>(xt + off);

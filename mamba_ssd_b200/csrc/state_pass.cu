@@ -58,60 +58,58 @@ __global__ void __launch_bounds__(256) state_pass_kernel(float *__restrict__ sta
     if (h_final) *reinterpret_cast<float4 *>(h_final + bh * PN + e) = s;
 }
 
-// Variant for the tensor-core chunk scan: the state each block starts from is emitted in bf16,
-// transposed to [N][P] (the row-major layout whose 128-byte-swizzled TMA tiles are the MN-major
-// B operand of O = C h_prev^T), into a separate buffer; h_final stays float32 [P][N].
-// Thread (n, p0..p0+7): 8 coalesced fp32 loads per block (consecutive n across lanes) and one
-// 16-byte store of 8 bf16.
-__global__ void __launch_bounds__(256) state_pass_t_kernel(const float *__restrict__ states,
-                                                           const float *__restrict__ acs,
+// Variant for the tensor-core path: the block states arrive transposed, S^T [N][P] fp32 (the
+// layout of the tcgen05 accumulator), and the state each block starts from is emitted in the
+// same transposed layout in bf16 -- row-major [N][P], whose 128-byte-swizzled TMA tiles are the
+// MN-major B operand of O = C h_prev^T -- into a separate buffer.  h0 and h_final keep the
+// public [P][N] float32 layout.  Thread (n, p0..p0+3): one float4 load and one 8-byte store
+// per block, consecutive threads walking p then n, so every warp access is contiguous.
+__global__ void __launch_bounds__(256) state_pass_t_kernel(const float *__restrict__ statesT,
+                                                           const float *__restrict__ acs2,
                                                            const float *__restrict__ h0,
                                                            float *__restrict__ h_final,
                                                            __nv_bfloat16 *__restrict__ hT, int H,
                                                            int P, int N, int nc, int Q) {
-    constexpr int kAhead = 4;
+    constexpr int kAhead = 8;
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    const int n = t % N, p0 = (t / N) * 8;
+    const int p0 = (t * 4) % P, n = (t * 4) / P;
     const int h = blockIdx.y, b = blockIdx.z;
-    if (p0 >= P) return;
+    if (n >= N) return;
     const size_t bh = (size_t)b * H + h;
     const size_t PN = (size_t)P * N;
-    float s[8];
+    float s[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) s[i] = h0 ? h0[bh * PN + (size_t)(p0 + i) * N + n] : 0.f;
-    const float *a_last = acs + bh * (size_t)nc * Q + (Q - 1);
+    for (int i = 0; i < 4; ++i) s[i] = h0 ? h0[bh * PN + (size_t)(p0 + i) * N + n] : 0.f;
+    const float *a_last = acs2 + bh * (size_t)nc * Q + (Q - 1);
+    const size_t off = (size_t)n * P + p0;
     for (int c0 = 0; c0 < nc; c0 += kAhead) {
-        float in[kAhead][8];
+        float4 in[kAhead];
         float a[kAhead];
 #pragma unroll
         for (int j = 0; j < kAhead; ++j) {
             if (c0 + j < nc) {
-                const float *src = states + (((size_t)b * nc + c0 + j) * H + h) * PN + n;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) in[j][i] = src[(size_t)(p0 + i) * N];
+                in[j] = *reinterpret_cast<const float4 *>(statesT + (((size_t)b * nc + c0 + j) * H + h) * PN + off);
                 a[j] = a_last[(size_t)(c0 + j) * Q];
             }
         }
 #pragma unroll
         for (int j = 0; j < kAhead; ++j) {
             if (c0 + j < nc) {
-                uint4 v;
-                uint32_t *u = reinterpret_cast<uint32_t *>(&v);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    __nv_bfloat162 p2 = __floats2bfloat162_rn(s[2 * i], s[2 * i + 1]);
-                    u[i] = *reinterpret_cast<uint32_t *>(&p2);
-                }
-                *reinterpret_cast<uint4 *>(hT + ((((size_t)b * nc + c0 + j) * H + h) * N + n) * P + p0) = v;
+                __nv_bfloat162 lo2 = __floats2bfloat162_rn(s[0], s[1]);
+                __nv_bfloat162 hi2 = __floats2bfloat162_rn(s[2], s[3]);
+                uint2 v = make_uint2(*reinterpret_cast<uint32_t *>(&lo2), *reinterpret_cast<uint32_t *>(&hi2));
+                *reinterpret_cast<uint2 *>(hT + (((size_t)b * nc + c0 + j) * H + h) * PN + off) = v;
                 const float d = exp2f(a[j]);  // acs arrives as acs * log2(e) on this path
-#pragma unroll
-                for (int i = 0; i < 8; ++i) s[i] = fmaf(d, s[i], in[j][i]);
+                s[0] = fmaf(d, s[0], in[j].x);
+                s[1] = fmaf(d, s[1], in[j].y);
+                s[2] = fmaf(d, s[2], in[j].z);
+                s[3] = fmaf(d, s[3], in[j].w);
             }
         }
     }
     if (h_final) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) h_final[bh * PN + (size_t)(p0 + i) * N + n] = s[i];
+        for (int i = 0; i < 4; ++i) h_final[bh * PN + (size_t)(p0 + i) * N + n] = s[i];
     }
 }
 
@@ -119,7 +117,7 @@ cudaError_t launch_state_pass_t(const float *states, const float *acs, const flo
                                 __nv_bfloat16 *hT, int B, int L, int H, int P, int N, int chunk,
                                 cudaStream_t st) {
     const int nc = cdiv(L, chunk);
-    dim3 grid(cdiv(P * N / 8, 256), H, B);
+    dim3 grid(cdiv(P * N / 4, 256), H, B);
     state_pass_t_kernel<<<grid, 256, 0, st>>>(states, acs, h0, h_final, hT, H, P, N, nc, chunk);
     return cudaGetLastError();
 }
