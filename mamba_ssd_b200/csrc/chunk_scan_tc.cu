@@ -13,24 +13,36 @@
 // block, head):
 //   CB  = C_k B_k^T                 once per (batch, block, group), kept in TMEM, fp32
 //   O   = C_k h_prev^T              h_prev^T arrives by TMA as a bf16 [n][p] tile
-//   P~  = mask(CB * dt_s * exp(acs_l - acs_s)) + D on the diagonal   (CUDA cores -> TMEM;
-//         dt_s exp(acs_l - acs_s) is one ex2 of precomputed per-token factors)
+//   P~  = mask(CB * dt_s * exp(acs_l - acs_s)) + D on the diagonal   (CUDA cores -> TMEM,
+//         from precomputed per-token factors colv = acs*log2(e) - log2(dt), acs2 = acs*log2(e))
 //   Y   = P~ x_k                    A operand read from TMEM, x_k straight from its TMA tile
 //   y_l = Y_l + exp(acs_l) O_l      (epilogue, fp32 -> bf16)
 // Folding dt into the columns of P~ and D into its diagonal means x is used as loaded:
-// no x operand is rewritten, and no x is re-read for the skip.  exp() is only ever taken of
-// a non-positive argument (masked before the exp), so nothing overflows.
+// no x operand is rewritten, and no x is re-read for the skip.
+//
+// The decay factor of P~ is formed per 32 x 32 sub-block.  Below the diagonal (rows in
+// sub-block r, columns in sub-block c < r) it factors through the cumsum at the last token
+// of column sub-block c:
+//   dt_s exp(acs_l - acs_s) = exp(acs_l - acs_ref) * dt_s exp(acs_ref - acs_s),
+// both factors at most 1 since acs is non-increasing, so a 32 x 32 sub-block costs 64
+// exponentials instead of 1024.  A diagonal sub-block factors through its middle token when
+// the cumsum falls by at most 96 (base 2) across it, so neither factor leaves fp32's range;
+// otherwise its factors are taken one by one.  Above the diagonal P~ is zero: those TMEM
+// columns are cleared once per CTA and never written again.
 //
 // Structure: persistent CTAs own contiguous ranges of items ordered (batch, block, head), so
-// consecutive items share the C/B tiles and CB.  Warp-specialised, the roles meeting only at
-// mbarriers:
-//   warp 0      TMA producer: C/B tiles per (batch, block, group); x tile, h_prev^T tile and
-//               the item's per-token factors into a ring of kStages stages
-//   warp 1      MMA issuer (one lane): CB per tile; O and Y per item into one of two TMEM sets
-//   warps 2..17 workers: P~ of item j into TMEM, then the epilogue of item j - 1
-// so the tensor core runs item j's products while the CUDA cores form item j+1's P~ and
-// write item j-1's outputs.
+// consecutive items share the C/B tiles and CB.  Warp-specialised, every role with its own
+// loop, the roles meeting only at mbarriers:
+//   warp 0       TMA producer: C/B tiles per (batch, block, group); x tile, h_prev^T tile and
+//                the item's per-token factors into a ring of kStages stages
+//   warp 1       MMA issuer (one lane): CB per tile; O and Y per item into one of two TMEM sets
+//   warps 2..9   P~ of an item into its TMEM set
+//   warps 10..17 epilogue: y = Y + exp(acs) O of an item into a swizzled shared-memory tile
+//                that one TMA store writes out (tokens past L are clipped by the store)
+// so the tensor core runs item j's products while P~ of item j+1 is formed and item j-1's
+// outputs are written.
 #include "common.cuh"
+#include "items.cuh"
 #include "launch.h"
 #include "tc.cuh"
 #include "tmap.h"
@@ -39,8 +51,8 @@ namespace ssd {
 
 namespace csc {
 constexpr int R = 128, P = 64, N = 128;
-constexpr int kWorkers = 16;
-constexpr int kThreads = (2 + kWorkers) * 32;
+constexpr int kPt = 8, kEpi = 8;
+constexpr int kThreads = (2 + kPt + kEpi) * 32;
 constexpr int kStages = 4;
 constexpr uint32_t kBox = R * 128;            // [128 rows][64 bf16] swizzled box: 16 KB
 constexpr uint32_t kOffC = 0;                 // C block: 2 n-boxes, 32 KB
@@ -48,32 +60,36 @@ constexpr uint32_t kOffB = 2 * kBox;          // B block: 2 n-boxes, 32 KB
 constexpr uint32_t kOffStage = 4 * kBox;      // ring of stages
 constexpr uint32_t kStX = 0, kStH = kBox, kStRows = 2 * kBox;  // x box, h_prev^T box, colv+acs2
 constexpr uint32_t kStageBytes = 2 * kBox + 2048;             // keeps 1024-byte alignment
-constexpr uint32_t kOffBar = kOffStage + kStages * kStageBytes;
+constexpr uint32_t kOffOut = kOffStage + kStages * kStageBytes;  // y staging [128][64] bf16
+constexpr uint32_t kOffVb = kOffOut + kBox;                       // per-warp column factors
+constexpr uint32_t kOffBar = kOffVb + kPt * 32 * 4;
 constexpr uint32_t kSmem = kOffBar + 256 + 1024;
 // TMEM columns: CB, then two sets of {P~ (bf16 pairs), Y, O}
 constexpr uint32_t kColCB = 0, kSet = 192, kSet0 = 128, kOffPT = 0, kOffY = 64, kOffO = 128;
 constexpr uint32_t kTmemCols = 512;
+constexpr float kDiagFactorRange = 96.f;
+constexpr int kEpiBar = 1;  // named barrier of the epilogue warps  // log2 range of a diagonal sub-block that is factored
 }  // namespace csc
 
 __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_h,
-    const float *__restrict__ dtf, const float *__restrict__ acs, const float *__restrict__ D,
-    __nv_bfloat16 *__restrict__ y, int *__restrict__ status, int L, int H, int G, int nk, int total) {
+    const __grid_constant__ CUtensorMap tm_y, const float *__restrict__ dtf, const float *__restrict__ acs,
+    const float *__restrict__ D, int *__restrict__ status, int H, int G, int nk, int total) {
     using namespace csc;
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
-    uint64_t *st_full = bars;                  // [kStages] TMA -> workers, MMA
+    uint64_t *st_full = bars;                  // [kStages] TMA -> P~, MMA
     uint64_t *st_empty = st_full + kStages;    // [kStages] MMA commit after Y -> producer
     uint64_t *ld_full = st_empty + kStages;    // C/B tiles landed
     uint64_t *ld_empty = ld_full + 1;          // MMA commit after the last O of a tile
     uint64_t *cb_full = ld_empty + 1;          // MMA commit after CB
-    uint64_t *cb_empty = cb_full + 1;          // workers done reading CB of a tile
-    uint64_t *pt_full = cb_empty + 1;          // [2] workers wrote P~ of a set
+    uint64_t *cb_empty = cb_full + 1;          // P~ warps done reading CB of a tile
+    uint64_t *pt_full = cb_empty + 1;          // [2] P~ warps wrote P~ of a set
     uint64_t *acc_full = pt_full + 2;          // [2] MMA commit after Y
-    uint64_t *acc_empty = acc_full + 2;        // [2] workers read Y, O of a set
+    uint64_t *acc_empty = acc_full + 2;        // [2] epilogue read Y, O of a set
     uint64_t *fin = acc_empty + 2;             // MMA commit after the last MMA of the CTA
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -82,7 +98,6 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
     const int first = (int)((long long)blockIdx.x * total / gridDim.x);
     const int cnt = (int)((long long)(blockIdx.x + 1) * total / gridDim.x) - first;
     if (cnt <= 0) return;
-    const int hpg = H / G;
     const size_t Lp = (size_t)nk * R;
 
     if (tid == 0) {
@@ -93,11 +108,11 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
         mbar_init(ld_full, 1);
         mbar_init(ld_empty, 1);
         mbar_init(cb_full, 1);
-        mbar_init(cb_empty, kWorkers);
+        mbar_init(cb_empty, kPt);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&pt_full[i], kWorkers);
+            mbar_init(&pt_full[i], kPt);
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], kWorkers);
+            mbar_init(&acc_empty[i], kEpi);
         }
         mbar_init(fin, 1);
         *abort_flag = 0;
@@ -106,6 +121,7 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
         tma_prefetch_desc(&tm_b);
         tma_prefetch_desc(&tm_c);
         tma_prefetch_desc(&tm_h);
+        tma_prefetch_desc(&tm_y);
     }
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
@@ -113,20 +129,6 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    auto item = [&](int j, int &b, int &k, int &h) {
-        const int it = first + j;
-        h = it % H;
-        const int t = it / H;
-        k = t % nk;
-        b = t / nk;
-    };
-    auto tile_key = [&](int j) {
-        int b, k, h;
-        item(j, b, k, h);
-        return (b * nk + k) * G + h / hpg;
-    };
-    auto new_tile = [&](int j) { return j == 0 || tile_key(j) != tile_key(j - 1); };
-    auto last_of_tile = [&](int j) { return j == cnt - 1 || tile_key(j + 1) != tile_key(j); };
     auto stage = [&](int j) { return smem + kOffStage + (uint32_t)(j % kStages) * kStageBytes; };
     // a bounded wait that gives up at once when another role has already timed out
     auto wait = [&](uint64_t *bar, uint32_t parity) {
@@ -142,27 +144,26 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
         if (lane == 0) {
+            ItemCursor it(first, H, G, nk);
             int tiles = 0;
-            for (int j = 0; j < cnt; ++j) {
-                int b, k, h;
-                item(j, b, k, h);
-                if (new_tile(j)) {
+            for (int j = 0; j < cnt; ++j, it.next()) {
+                const int h = it.h();
+                if (j == 0 || it.tile_first()) {
                     if (tiles > 0 && !wait(ld_empty, (tiles - 1) & 1)) break;
-                    const int g = h / hpg;
                     mbar_arrive_expect_tx(ld_full, 4 * kBox);
-                    tma_load_3d(smem + kOffC, &tm_c, g * N, k * R, b, ld_full);
-                    tma_load_3d(smem + kOffC + kBox, &tm_c, g * N + 64, k * R, b, ld_full);
-                    tma_load_3d(smem + kOffB, &tm_b, g * N, k * R, b, ld_full);
-                    tma_load_3d(smem + kOffB + kBox, &tm_b, g * N + 64, k * R, b, ld_full);
+                    tma_load_3d(smem + kOffC, &tm_c, it.g * N, it.k * R, it.b, ld_full);
+                    tma_load_3d(smem + kOffC + kBox, &tm_c, it.g * N + 64, it.k * R, it.b, ld_full);
+                    tma_load_3d(smem + kOffB, &tm_b, it.g * N, it.k * R, it.b, ld_full);
+                    tma_load_3d(smem + kOffB + kBox, &tm_b, it.g * N + 64, it.k * R, it.b, ld_full);
                     ++tiles;
                 }
                 const int s = j % kStages;
                 if (j >= kStages && !wait(&st_empty[s], ((j / kStages) - 1) & 1)) break;
                 uint8_t *st = stage(j);
-                const size_t row = ((size_t)b * H + h) * Lp + (size_t)k * R;
+                const size_t row = ((size_t)it.b * H + h) * Lp + (size_t)it.k * R;
                 mbar_arrive_expect_tx(&st_full[s], 2 * kBox + 2 * R * 4);
-                tma_load_3d(st + kStX, &tm_x, h * P, k * R, b, &st_full[s]);
-                tma_load_2d(st + kStH, &tm_h, 0, (int)((((size_t)b * nk + k) * H + h) * N), &st_full[s]);
+                tma_load_3d(st + kStX, &tm_x, h * P, it.k * R, it.b, &st_full[s]);
+                tma_load_2d(st + kStH, &tm_h, 0, (int)((((size_t)it.b * nk + it.k) * H + h) * N), &st_full[s]);
                 bulk_load(st + kStRows, dtf + row, R * 4, &st_full[s]);
                 bulk_load(st + kStRows + R * 4, acs + row, R * 4, &st_full[s]);
             }
@@ -172,20 +173,21 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
         if (lane == 0) {
             constexpr uint32_t id_cb = idesc_bf16_f32(128, 128, false, false);
             constexpr uint32_t id_kmn = idesc_bf16_f32(128, 64, false, true);  // K-major A, MN-major B
-            const uint32_t c0 = smem_u32(smem + kOffC), b0 = smem_u32(smem + kOffB);
+            const uint64_t dc = desc_kmajor_sw128(smem_u32(smem + kOffC));
+            const uint64_t db = desc_kmajor_sw128(smem_u32(smem + kOffB));
+            ItemCursor it(first, H, G, nk);
             int tiles = 0;
-            for (int j = 0; j < cnt; ++j) {
+            for (int j = 0; j < cnt; ++j, it.next()) {
                 const int s = j % kStages, t = j & 1;
                 const uint32_t set = tmem + kSet0 + t * kSet;
-                if (new_tile(j)) {  // CB = C B^T, once the workers are done with the previous CB
+                if (j == 0 || it.tile_first()) {  // CB = C B^T, once P~ is done with the previous CB
                     if (!wait(ld_full, tiles & 1)) break;
                     if (tiles > 0 && !wait(cb_empty, (tiles - 1) & 1)) break;
                     tc_fence_after();
-#pragma unroll 1
+#pragma unroll
                     for (int kk = 0; kk < N / 16; ++kk) {
                         const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                        mma_ss(tmem + kColCB, desc_kmajor_sw128(c0 + off), desc_kmajor_sw128(b0 + off), id_cb,
-                               kk > 0 ? 1u : 0u);
+                        mma_ss(tmem + kColCB, desc_add(dc, off), desc_add(db, off), id_cb, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(cb_full);
                     ++tiles;
@@ -193,93 +195,92 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
                 if (!wait(&st_full[s], (j / kStages) & 1)) break;
                 if (j >= 2 && !wait(&acc_empty[t], ((j >> 1) - 1) & 1)) break;
                 tc_fence_after();
-                const uint32_t hb = smem_u32(stage(j) + kStH), xb = smem_u32(stage(j) + kStX);
-#pragma unroll 1
+                const uint64_t dh = desc_mnmajor_sw128(smem_u32(stage(j) + kStH), kBox);
+                const uint64_t dx = desc_mnmajor_sw128(smem_u32(stage(j) + kStX), kBox);
+#pragma unroll
                 for (int kk = 0; kk < N / 16; ++kk)  // O = C h_prev^T
-                    mma_ss(set + kOffO, desc_kmajor_sw128(c0 + (kk >> 2) * kBox + (kk & 3) * 32),
-                           desc_mnmajor_sw128(hb + kk * 2048, kBox), id_kmn, kk > 0 ? 1u : 0u);
+                    mma_ss(set + kOffO, desc_add(dc, (kk >> 2) * kBox + (kk & 3) * 32), desc_add(dh, kk * 2048),
+                           id_kmn, kk > 0 ? 1u : 0u);
                 if (!wait(&pt_full[t], (j >> 1) & 1)) break;
                 tc_fence_after();
-#pragma unroll 1
+#pragma unroll
                 for (int kk = 0; kk < R / 16; ++kk)  // Y = P~ x
-                    mma_ts(set + kOffY, set + kOffPT + kk * 8, desc_mnmajor_sw128(xb + kk * 2048, kBox), id_kmn,
-                           kk > 0 ? 1u : 0u);
+                    mma_ts(set + kOffY, set + kOffPT + kk * 8, desc_add(dx, kk * 2048), id_kmn, kk > 0 ? 1u : 0u);
                 mma_commit(&acc_full[t]);
                 mma_commit(&st_empty[s]);
-                if (last_of_tile(j)) mma_commit(ld_empty);
+                if (j == cnt - 1 || it.tile_last()) mma_commit(ld_empty);
             }
             // every MMA (and every arrive it triggers) has landed before TMEM is released
             mma_commit(fin);
             mbar_wait(fin, 0, status);
         }
-    } else {
-        // ---------------------------------------------------------------- workers
-        // warps w, w + 4, w + 8, w + 12 share TMEM lanes 32 (w % 4) .. + 31 (rows of the
-        // block); the four split P~'s 32-column blocks and the 16-column output quarters
-        const int rq = warp & 3, cq = (warp - 2) >> 2;
+    } else if (warp < 2 + kPt) {
+        // ---------------------------------------------------------------- P~
+        // TMEM lanes 32 (warp % 4) .. + 31 are rows rq of the block; this warp forms the
+        // 32-column sub-blocks pc and 3 - pc of those rows (those above the diagonal are zero)
+        const int rq = warp & 3, pc = (warp - 2) >> 2;
         const int myrow = rq * 32 + lane;
         const uint32_t lane_base = (uint32_t)(rq * 32) << 16;
-        auto epilogue = [&](int j, float scale) {
-            const int t = j & 1;
-            if (!wait(&acc_full[t], (j >> 1) & 1)) return false;
-            tc_fence_after();
-            int b, k, h;
-            item(j, b, k, h);
-            const uint32_t set = tmem + lane_base + kSet0 + t * kSet;
-            float yv[16], ov[16];
-            tmem_ld16(set + kOffY + cq * 16, yv);
-            tmem_ld16(set + kOffO + cq * 16, ov);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[t]);
-            const int tok = k * R + myrow;
-            if (tok < L) {
-                uint4 *yr = reinterpret_cast<uint4 *>(y + (((size_t)b * L + tok) * H + h) * P + cq * 16);
+        float *vb = reinterpret_cast<float *>(smem + kOffVb) + (warp - 2) * 32;
+        {
+            uint32_t zero[16];
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    uint32_t o[4];
+            for (int i = 0; i < 16; ++i) zero[i] = 0u;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int e = q * 8 + 2 * i;
-                        o[i] = pack_bf16x2(fmaf(scale, ov[e], yv[e]), fmaf(scale, ov[e + 1], yv[e + 1]));
-                    }
-                    yr[q] = make_uint4(o[0], o[1], o[2], o[3]);
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int bi = 0; bi < 2; ++bi) {
+                    const int cb = bi == 0 ? pc : 3 - pc;
+                    if (cb > rq) tmem_st16(tmem + lane_base + kSet0 + t * kSet + kOffPT + cb * 16, zero);
                 }
-            }
-            return true;
-        };
+        }
+        ItemCursor it(first, H, G, nk);
         int tiles = 0;
-        float scale_prev = 0.f;
-        for (int j = 0; j < cnt; ++j) {
+        for (int j = 0; j < cnt; ++j, it.next()) {
             const int s = j % kStages, t = j & 1;
-            if (new_tile(j)) {
-                if (!wait(cb_full, tiles & 1)) break;
+            if (j == 0 || it.tile_first()) {
+                if (!__all_sync(0xffffffffu, wait(cb_full, tiles & 1))) break;
                 ++tiles;
             }
-            if (!wait(&st_full[s], (j / kStages) & 1)) break;
+            bool ok = wait(&st_full[s], (j / kStages) & 1);
+            // P~ of this set was last read by the MMA of item j - 2
+            if (ok && j >= 2) ok = wait(&acc_full[t], ((j >> 1) - 1) & 1);
+            if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform
             tc_fence_after();
-            int b, k, h;
-            item(j, b, k, h);
-            // P~ = mask(CB * 2^(acs2_l - colv_s)) + D on the diagonal, colv = acs2 - log2(dt):
-            // dt_s exp(acs_l - acs_s) = 2^(acs2_l - colv_s)
             const float *colv = reinterpret_cast<const float *>(stage(j) + kStRows);
             const float *acs2 = colv + R;
             const float al = acs2[myrow];
-            const float d = D ? __ldg(D + h) : 0.f;
-            const uint32_t set = tmem + kSet0 + t * kSet;
-            {
-                const int blk = cq;  // one 32-column block of P~ per warp
-                uint32_t packed[16];
-                if (blk > rq) {  // entirely above the diagonal for these rows
+            const float d = D ? __ldg(D + it.h()) : 0.f;
+            const uint32_t set = tmem + lane_base + kSet0 + t * kSet;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) packed[i] = 0u;
-                } else {
-                    float v[32];
-                    tmem_ld16(tmem + lane_base + kColCB + blk * 32, *reinterpret_cast<float(*)[16]>(&v[0]));
-                    tmem_ld16(tmem + lane_base + kColCB + blk * 32 + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+            for (int bi = 0; bi < 2; ++bi) {
+                const int cb = bi == 0 ? pc : 3 - pc;
+                if (cb > rq) continue;  // warp-uniform
+                float v[32];
+                tmem_ld16(tmem + lane_base + kColCB + cb * 32, *reinterpret_cast<float(*)[16]>(&v[0]));
+                tmem_ld16(tmem + lane_base + kColCB + cb * 32 + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+                const bool diag = cb == rq;
+                const bool factored = !diag || acs2[cb * 32] - acs2[cb * 32 + 31] <= kDiagFactorRange;
+                if (factored) {
+                    // P~_ls = CB_ls * 2^(acs2_l - ref) * 2^(ref - colv_s); colv = acs2 - log2(dt)
+                    const float ref = diag ? acs2[cb * 32 + 15] : acs2[cb * 32 + 31];
+                    vb[lane] = ex2_approx(ref - colv[cb * 32 + lane]);
+                    __syncwarp();
+                    const float u = ex2_approx(al - ref);
                     tmem_wait_ld();
-                    const float4 *c4 = reinterpret_cast<const float4 *>(colv + blk * 32);
+                    const float4 *v4 = reinterpret_cast<const float4 *>(vb);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 c = v4[i];
+                        v[4 * i + 0] *= u * c.x;
+                        v[4 * i + 1] *= u * c.y;
+                        v[4 * i + 2] *= u * c.z;
+                        v[4 * i + 3] *= u * c.w;
+                    }
+                    __syncwarp();
+                } else {
+                    tmem_wait_ld();
+                    const float4 *c4 = reinterpret_cast<const float4 *>(colv + cb * 32);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const float4 c = c4[i];
@@ -288,28 +289,70 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
                         v[4 * i + 2] *= ex2_approx(al - c.z);
                         v[4 * i + 3] *= ex2_approx(al - c.w);
                     }
-                    if (blk == rq) {  // the diagonal block: causal mask and the D skip
-                        const int ld = myrow - blk * 32;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = i < ld ? v[i] : (i == ld ? v[i] + d : 0.f);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
                 }
-                tmem_st16(set + lane_base + kOffPT + blk * 16, packed);
+                if (diag) {  // causal mask and the D skip; a select, so what lies above is dropped
+                    const int ld = myrow - cb * 32;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = i < ld ? v[i] : (i == ld ? v[i] + d : 0.f);
+                }
+                uint32_t packed[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                tmem_st16(set + kOffPT + cb * 16, packed);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&pt_full[t]);
-                if (last_of_tile(j)) mbar_arrive(cb_empty);
+                if (j == cnt - 1 || it.tile_last()) mbar_arrive(cb_empty);
             }
-            const float scale_j = ex2_approx(al);  // exp(acs_l) for item j's epilogue
-            if (j >= 1 && !epilogue(j - 1, scale_prev)) break;
-            scale_prev = scale_j;
         }
-        if (!*abort_flag) epilogue(cnt - 1, scale_prev);
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        const int rq = warp & 3, half = (warp - 2 - kPt) >> 2;  // TMEM lane quarter, 32 columns
+        const int myrow = rq * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(rq * 32) << 16;
+        const bool leader = warp == 2 + kPt && lane == 0;  // issues the stores
+        ItemCursor it(first, H, G, nk);
+        for (int j = 0; j < cnt; ++j, it.next()) {
+            const int t = j & 1, h = it.h();
+            // exp(acs_l) from the log2-form cumsum; read here, the stage may be refilled by now
+            const float al = __ldg(acs + ((size_t)it.b * H + h) * Lp + (size_t)it.k * R + myrow);
+            const bool ok = __all_sync(0xffffffffu, wait(&acc_full[t], (j >> 1) & 1));
+            uint32_t o[16];
+            if (ok) {
+                tc_fence_after();
+                const uint32_t set = tmem + lane_base + kSet0 + t * kSet;
+                float yv[32], ov[32];
+                tmem_ld16(set + kOffY + half * 32, *reinterpret_cast<float(*)[16]>(&yv[0]));
+                tmem_ld16(set + kOffY + half * 32 + 16, *reinterpret_cast<float(*)[16]>(&yv[16]));
+                tmem_ld16(set + kOffO + half * 32, *reinterpret_cast<float(*)[16]>(&ov[0]));
+                tmem_ld16(set + kOffO + half * 32 + 16, *reinterpret_cast<float(*)[16]>(&ov[16]));
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[t]);
+                const float scale = ex2_approx(al);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    o[i] = pack_bf16x2(fmaf(scale, ov[2 * i], yv[2 * i]), fmaf(scale, ov[2 * i + 1], yv[2 * i + 1]));
+            }
+            // the staging tile is free once the previous item's store has read it
+            if (leader) bulk_wait_read();
+            if (!named_barrier_and(kEpiBar, kEpi * 32, ok)) break;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4 *>(smem + kOffOut + sw128_offset(myrow, half * 4 + q)) =
+                    make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+            fence_proxy_async_smem();
+            named_barrier(kEpiBar, kEpi * 32);
+            if (leader) {
+                tma_store_3d(&tm_y, smem + kOffOut, h * P, it.k * R, it.b);
+                bulk_commit();
+            }
+        }
+        if (leader) bulk_wait_all();
     }
 
     __syncthreads();
@@ -330,7 +373,7 @@ cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, 
     using namespace csc;
     const int nk = cdiv(L, R);
     const int total = B * nk * H;
-    CUtensorMap tm_x, tm_b, tm_c, tm_h;
+    CUtensorMap tm_x, tm_b, tm_c, tm_h, tm_y;
     cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B,
                                       (uint64_t)H * P * 2, (uint64_t)L * H * P * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
@@ -342,10 +385,13 @@ cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, 
     if (e != cudaSuccess) return e;
     e = make_tmap_bf16_2d(&tm_h, hT, (uint64_t)P, (uint64_t)B * nk * H * N, (uint64_t)P * 2, 64, R);
     if (e != cudaSuccess) return e;
+    e = make_tmap_bf16_3d(&tm_y, y, (uint64_t)H * P, (uint64_t)L, (uint64_t)B, (uint64_t)H * P * 2,
+                          (uint64_t)L * H * P * 2, 64, R, 1);
+    if (e != cudaSuccess) return e;
     const int grid = total < num_sms ? total : num_sms;
     cudaFuncSetAttribute(chunk_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
-    chunk_scan_tc_kernel<<<grid, kThreads, kSmem, st>>>(tm_x, tm_b, tm_c, tm_h, dtf, acs, D,
-                                                        (__nv_bfloat16 *)y, status, L, H, G, nk, total);
+    chunk_scan_tc_kernel<<<grid, kThreads, kSmem, st>>>(tm_x, tm_b, tm_c, tm_h, tm_y, dtf, acs, D, status, H, G,
+                                                        nk, total);
     return cudaGetLastError();
 }
 

@@ -20,14 +20,17 @@
 //
 // Structure: persistent CTAs, one per SM, each owning a contiguous range of (batch, block,
 // head) items (consecutive items share the block's B tile).  Warp-specialised:
-//   warp 0      TMA producer: B tile per (batch, block, group); x tile + the item's
-//               per-token factors into a ring of kStages stages
-//   warp 1      MMA issuer (one lane): 16 MMAs per item into one of two TMEM accumulators
-//   warps 2..17 workers: scale rows by w into hi (in place) and lo; drain the accumulator of
-//               the item before to global memory (the state is written transposed, [N][P])
-// The roles meet only at mbarriers (full/empty per stage, per accumulator, per B tile), so
-// the tensor core runs back to back while the workers transform and drain other items.
+//   warp 0       TMA producer: B tile per (batch, block, group); x tile + the item's
+//                per-token factors into a ring of kStages stages
+//   warp 1       MMA issuer (one lane): 16 MMAs per item into one of two TMEM accumulators
+//   warps 2..9   transform: scale rows by w into hi (in place) and lo
+//   warps 10..17 epilogue: drain an accumulator through a swizzled shared-memory tile that
+//                one TMA store per 32-column half writes out (S^T, [N][P], fp32)
+// Every role runs its own loop and the roles meet only at mbarriers (full/empty per stage,
+// per accumulator, per B tile), so the tensor core, the transform of the next item and the
+// drain of the previous one overlap.
 #include "common.cuh"
+#include "items.cuh"
 #include "launch.h"
 #include "tc.cuh"
 #include "tmap.h"
@@ -36,32 +39,34 @@ namespace ssd {
 
 namespace cst {
 constexpr int R = 128, P = 64, N = 128;
-constexpr int kWorkers = 16;
-constexpr int kThreads = (2 + kWorkers) * 32;
+constexpr int kXform = 8, kEpi = 8;
+constexpr int kThreads = (2 + kXform + kEpi) * 32;
 constexpr int kStages = 4;
 constexpr uint32_t kBox = R * 128;                 // [128 rows][64 bf16], 16 KB
 constexpr uint32_t kOffB = 0;                      // B block: 2 n-boxes, 32 KB
 constexpr uint32_t kStageBytes = 2 * kBox + 1024;  // x/hi box, lo box, colv[128] + acs2[128]
 constexpr uint32_t kOffStage = 2 * kBox;
-constexpr uint32_t kOffBar = kOffStage + kStages * kStageBytes;
+constexpr uint32_t kOffOut = kOffStage + kStages * kStageBytes;  // S^T staging: 2 x [128][32] fp32
+constexpr uint32_t kOffBar = kOffOut + 2 * kBox;
+constexpr int kEpiBar = 1;  // named barrier of the epilogue warps
 constexpr uint32_t kSmem = kOffBar + 256 + 1024;  // + slack for 1024-byte alignment
 constexpr uint32_t kTmemCols = 128;               // two 64-column fp32 accumulators
 }  // namespace cst
 
 __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-    const float *__restrict__ dtf, const float *__restrict__ acs, float *__restrict__ states,
+    const __grid_constant__ CUtensorMap tm_s, const float *__restrict__ dtf, const float *__restrict__ acs,
     int *__restrict__ status, int H, int G, int nk, int total) {
     using namespace cst;
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
-    uint64_t *st_full = bars;                 // [kStages] TMA -> workers
-    uint64_t *op_full = st_full + kStages;    // [kStages] workers -> MMA (operands written)
+    uint64_t *st_full = bars;                 // [kStages] TMA -> transform
+    uint64_t *op_full = st_full + kStages;    // [kStages] transform -> MMA (operands written)
     uint64_t *st_empty = op_full + kStages;   // [kStages] MMA commit -> producer
-    uint64_t *acc_full = st_empty + kStages;  // [2] MMA commit -> workers
-    uint64_t *acc_empty = acc_full + 2;       // [2] workers -> MMA
+    uint64_t *acc_full = st_empty + kStages;  // [2] MMA commit -> epilogue
+    uint64_t *acc_empty = acc_full + 2;       // [2] epilogue -> MMA
     uint64_t *b_full = acc_empty + 2;         // B tile landed
     uint64_t *b_empty = b_full + 1;           // MMA commit after the last item of a tile
     uint64_t *fin = b_empty + 1;              // MMA commit after the last MMA of the CTA
@@ -72,18 +77,17 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     const int first = (int)((long long)blockIdx.x * total / gridDim.x);
     const int cnt = (int)((long long)(blockIdx.x + 1) * total / gridDim.x) - first;
     if (cnt <= 0) return;
-    const int hpg = H / G;
     const size_t Lp = (size_t)nk * R;
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&st_full[i], 1);
-            mbar_init(&op_full[i], kWorkers);
+            mbar_init(&op_full[i], kXform);
             mbar_init(&st_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], kWorkers);
+            mbar_init(&acc_empty[i], kEpi);
         }
         mbar_init(b_full, 1);
         mbar_init(b_empty, 1);
@@ -92,6 +96,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
         fence_barrier_init();
         tma_prefetch_desc(&tm_x);
         tma_prefetch_desc(&tm_b);
+        tma_prefetch_desc(&tm_s);
     }
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
@@ -99,30 +104,14 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    auto item = [&](int j, int &b, int &k, int &h) {
-        const int it = first + j;
-        h = it % H;
-        const int t = it / H;
-        k = t % nk;
-        b = t / nk;
-    };
-    auto b_key = [&](int j) {
-        int b, k, h;
-        item(j, b, k, h);
-        return (b * nk + k) * G + h / hpg;
-    };
-    auto new_tile = [&](int j) { return j == 0 || b_key(j) != b_key(j - 1); };
-    auto last_of_tile = [&](int j) { return j == cnt - 1 || b_key(j + 1) != b_key(j); };
     auto stage = [&](int j) { return smem + kOffStage + (uint32_t)(j % kStages) * kStageBytes; };
     // a bounded wait that gives up at once when another role has already timed out
     auto wait = [&](uint64_t *bar, uint32_t parity) {
-        while (!mbar_test(bar, parity)) {
-            if (*abort_flag) return false;
-            if (!mbar_wait(bar, parity, status)) {
-                *abort_flag = 1;
-                return false;
-            }
-            return true;
+        if (mbar_test(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (!mbar_wait(bar, parity, status)) {
+            *abort_flag = 1;
+            return false;
         }
         return true;
     };
@@ -130,24 +119,23 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
         if (lane == 0) {
+            ItemCursor it(first, H, G, nk);
             int tiles = 0;
-            for (int j = 0; j < cnt; ++j) {
-                int b, k, h;
-                item(j, b, k, h);
-                if (new_tile(j)) {
+            for (int j = 0; j < cnt; ++j, it.next()) {
+                const int h = it.h();
+                if (j == 0 || it.tile_first()) {
                     if (tiles > 0 && !wait(b_empty, (tiles - 1) & 1)) break;
                     mbar_arrive_expect_tx(b_full, 2 * kBox);
-                    const int g = h / hpg;
-                    tma_load_3d(smem + kOffB, &tm_b, g * N, k * R, b, b_full);
-                    tma_load_3d(smem + kOffB + kBox, &tm_b, g * N + 64, k * R, b, b_full);
+                    tma_load_3d(smem + kOffB, &tm_b, it.g * N, it.k * R, it.b, b_full);
+                    tma_load_3d(smem + kOffB + kBox, &tm_b, it.g * N + 64, it.k * R, it.b, b_full);
                     ++tiles;
                 }
                 const int s = j % kStages;
                 if (j >= kStages && !wait(&st_empty[s], ((j / kStages) - 1) & 1)) break;
                 uint8_t *st = stage(j);
-                const size_t row = ((size_t)b * H + h) * Lp + (size_t)k * R;
+                const size_t row = ((size_t)it.b * H + h) * Lp + (size_t)it.k * R;
                 mbar_arrive_expect_tx(&st_full[s], kBox + 2 * R * 4);
-                tma_load_3d(st, &tm_x, h * P, k * R, b, &st_full[s]);
+                tma_load_3d(st, &tm_x, h * P, it.k * R, it.b, &st_full[s]);
                 bulk_load(st + 2 * kBox, dtf + row, R * 4, &st_full[s]);
                 bulk_load(st + 2 * kBox + R * 4, acs + row, R * 4, &st_full[s]);
             }
@@ -156,76 +144,51 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(128, 64, true, true);
-            const uint32_t a0 = smem_u32(smem + kOffB);
+            const uint64_t da = desc_mnmajor_sw128(smem_u32(smem + kOffB), kBox);
+            ItemCursor it(first, H, G, nk);
             int tiles = 0;
-            for (int j = 0; j < cnt; ++j) {
+            for (int j = 0; j < cnt; ++j, it.next()) {
                 const int s = j % kStages, a = j & 1;
-                if (new_tile(j)) {
+                if (j == 0 || it.tile_first()) {
                     if (!wait(b_full, tiles & 1)) break;
                     ++tiles;
                 }
                 if (!wait(&op_full[s], (j / kStages) & 1)) break;
                 if (j >= 2 && !wait(&acc_empty[a], ((j >> 1) - 1) & 1)) break;
                 tc_fence_after();
-                uint8_t *st = stage(j);
-                const uint32_t bh = smem_u32(st), bl = smem_u32(st + kBox);
+                const uint64_t dh = desc_mnmajor_sw128(smem_u32(stage(j)), kBox), dl = desc_add(dh, kBox);
                 const uint32_t d = tmem + (uint32_t)(a * 64);
-#pragma unroll 1
+#pragma unroll
                 for (int kk = 0; kk < R / 16; ++kk)
-                    mma_ss(d, desc_mnmajor_sw128(a0 + kk * 2048, kBox), desc_mnmajor_sw128(bh + kk * 2048, kBox),
-                           idesc, kk > 0 ? 1u : 0u);
-#pragma unroll 1
-                for (int kk = 0; kk < R / 16; ++kk)
-                    mma_ss(d, desc_mnmajor_sw128(a0 + kk * 2048, kBox), desc_mnmajor_sw128(bl + kk * 2048, kBox),
-                           idesc, 1u);
+                    mma_ss(d, desc_add(da, kk * 2048), desc_add(dh, kk * 2048), idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < R / 16; ++kk) mma_ss(d, desc_add(da, kk * 2048), desc_add(dl, kk * 2048), idesc, 1u);
                 mma_commit(&acc_full[a]);
                 mma_commit(&st_empty[s]);
-                if (last_of_tile(j)) mma_commit(b_empty);
+                if (j == cnt - 1 || it.tile_last()) mma_commit(b_empty);
             }
             // every MMA (and every arrive it triggers) has landed before TMEM is released
             mma_commit(fin);
             mbar_wait(fin, 0, status);
         }
-    } else {
-        // ---------------------------------------------------------------- workers
-        const int wk = warp - 2;  // 0..15: rows [8 wk, 8 wk + 8) of the transform
-        const int quarter = warp & 3, colq = wk >> 2;  // epilogue: TMEM lane quarter, column quarter
-        auto epilogue = [&](int j) {
-            const int a = j & 1;
-            if (!wait(&acc_full[a], (j >> 1) & 1)) return false;
-            tc_fence_after();
-            int b, k, h;
-            item(j, b, k, h);
-            // S^T[n][p] row n = this lane, 16 columns: 64 contiguous bytes
-            float *out = states + (((size_t)b * nk + k) * H + h) * (size_t)(P * N) +
-                         (size_t)(quarter * 32 + lane) * P + colq * 16;
-            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 64 + colq * 16);
-            float v0[16];
-            tmem_ld16(taddr, v0);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[a]);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                reinterpret_cast<float4 *>(out)[q] = make_float4(v0[4 * q], v0[4 * q + 1], v0[4 * q + 2], v0[4 * q + 3]);
-            return true;
-        };
+    } else if (warp < 2 + kXform) {
+        // ---------------------------------------------------------------- transform
+        const int tw = warp - 2;  // rows [16 tw, 16 tw + 16)
         for (int j = 0; j < cnt; ++j) {
             const int s = j % kStages;
-            if (!wait(&st_full[s], (j / kStages) & 1)) break;
+            if (!__all_sync(0xffffffffu, wait(&st_full[s], (j / kStages) & 1))) break;  // warp-uniform
             uint8_t *xt = stage(j);
             uint8_t *lo = xt + kBox;
             const float *colv = reinterpret_cast<const float *>(xt + 2 * kBox);
             const float *acs2 = colv + R;
-            // w_s = dt_s exp(acs_last - acs_s) = exp2(acs2_last - colv_s); lanes 0..7 hold the
-            // weights of this warp's 8 rows
-            const float wl = lane < 8 ? ex2_approx(acs2[R - 1] - colv[wk * 8 + lane]) : 0.f;
+            // w_s = dt_s exp(acs_last - acs_s) = exp2(acs2_last - colv_s); lanes 0..15 hold the
+            // weights of this warp's 16 rows
+            const float wl = lane < 16 ? ex2_approx(acs2[R - 1] - colv[tw * 16 + lane]) : 0.f;
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {  // 8 rows x 8 chunks = 64 chunks over 32 lanes
+            for (int q = 0; q < 4; ++q) {  // 16 rows x 8 chunks = 128 chunks over 32 lanes
                 const int idx = q * 32 + lane;
                 const int rl = idx >> 3, chunk = idx & 7;
-                const int row = wk * 8 + rl;
+                const int row = tw * 16 + rl;
                 const float w = __shfl_sync(0xffffffffu, wl, rl);
                 const uint32_t off = sw128_offset(row, chunk);
                 uint4 raw = *reinterpret_cast<const uint4 *>(xt + off);
@@ -247,9 +210,46 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&op_full[s]);
-            if (j >= 1 && !epilogue(j - 1)) break;
         }
-        if (!*abort_flag) epilogue(cnt - 1);
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        // TMEM lane quarter (warp % 4) = rows n, column half = p range of 32
+        const int quarter = warp & 3, half = (warp - 2 - kXform) >> 2;
+        const int n = quarter * 32 + lane;
+        const bool leader = warp == 2 + kXform && lane == 0;  // issues the stores
+        uint8_t *box = smem + kOffOut + half * kBox;
+        ItemCursor it(first, H, G, nk);
+        for (int j = 0; j < cnt; ++j, it.next()) {
+            const int a = j & 1;
+            const bool ok = __all_sync(0xffffffffu, wait(&acc_full[a], (j >> 1) & 1));
+            float v[32];
+            if (ok) {
+                tc_fence_after();
+                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 64 + half * 32);
+                tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(&v[0]));
+                tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[a]);
+            }
+            // the staging tile is free once the previous item's stores have read it
+            if (leader) bulk_wait_read();
+            if (!named_barrier_and(kEpiBar, kEpi * 32, ok)) break;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<float4 *>(box + sw128_offset(n, c)) =
+                    make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            fence_proxy_async_smem();
+            named_barrier(kEpiBar, kEpi * 32);
+            if (leader) {
+                const int row = (int)((((size_t)it.b * nk + it.k) * H + it.h()) * N);
+                tma_store_2d(&tm_s, smem + kOffOut, 0, row);
+                tma_store_2d(&tm_s, smem + kOffOut + kBox, 32, row);
+                bulk_commit();
+            }
+        }
+        if (leader) bulk_wait_all();
     }
 
     __syncthreads();
@@ -274,16 +274,19 @@ cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const float *dt
     using namespace cst;
     const int nk = cdiv(L, R);
     const int total = B * nk * H;
-    CUtensorMap tm_x, tm_b;
+    CUtensorMap tm_x, tm_b, tm_s;
     cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B,
                                       (uint64_t)H * P * 2, (uint64_t)L * H * P * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
     e = make_tmap_bf16_3d(&tm_b, Bm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)G * N * 2,
                           (uint64_t)L * G * N * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
+    // S^T of every item as rows of 64 fp32: TMA boxes of 32 columns x 128 rows
+    e = make_tmap_f32_2d(&tm_s, states, (uint64_t)P, (uint64_t)total * N, (uint64_t)P * 4, 32, R);
+    if (e != cudaSuccess) return e;
     const int grid = total < num_sms ? total : num_sms;
     cudaFuncSetAttribute(chunk_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
-    chunk_state_tc_kernel<<<grid, kThreads, kSmem, st>>>(tm_x, tm_b, dtf, acs, states, status, H, G, nk,
+    chunk_state_tc_kernel<<<grid, kThreads, kSmem, st>>>(tm_x, tm_b, tm_s, dtf, acs, status, H, G, nk,
                                                          total);
     return cudaGetLastError();
 }

@@ -18,4 +18,9 @@ cudaError_t make_tmap_bf16_3d(CUtensorMap *out, const void *base, uint64_t d0, u
 cudaError_t make_tmap_bf16_2d(CUtensorMap *out, const void *base, uint64_t d0, uint64_t d1,
                               uint64_t stride1_bytes, uint32_t box0, uint32_t box1);
 
+// A 2-D fp32 tensor map with 128-byte swizzle: dims d0 (inner), d1; byte stride of dim 1
+// (box0 * 4 bytes must be <= 128 for the swizzle).
+cudaError_t make_tmap_f32_2d(CUtensorMap *out, const void *base, uint64_t d0, uint64_t d1,
+                             uint64_t stride1_bytes, uint32_t box0, uint32_t box1);
+
 }  // namespace ssd
