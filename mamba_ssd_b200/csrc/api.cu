@@ -197,14 +197,10 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
         const int blk = ssd::kTcBlock;
         ssd::PrefillWorkspace ws = ssd::carve_prefill_workspace(workspace, B, L, H, P, N, blk, true);
         if (L > 0) {
-            e = timed_launch(K_DECAY, st, [&] {
-                return ssd::launch_decay_prep(dtype, dt, A_log, dt_bias, dt_min, dt_max, ws.dtf, ws.acs,
-                                              ws.status, B, L, H, blk, true, st);
-            });
-            if (e != cudaSuccess) return cuda_status(e);
+            // the state kernel also forms the decay factors (step a1) of the items it owns
             e = timed_launch(K_STATE, st, [&] {
-                return ssd::launch_chunk_state_tc(x, Bm, ws.dtf, ws.acs, ws.states, ws.status, B, L, H, G,
-                                                  sm_count(), st);
+                return ssd::launch_chunk_state_tc(x, Bm, dt, A_log, dt_bias, dt_min, dt_max, ws.dtf, ws.acs,
+                                                  ws.states, ws.status, B, L, H, G, sm_count(), st);
             });
             if (e != cudaSuccess) return cuda_status(e);
         }
@@ -226,7 +222,7 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
     if (L > 0) {
         e = timed_launch(K_DECAY, st, [&] {
             return ssd::launch_decay_prep(dtype, dt, A_log, dt_bias, dt_min, dt_max, ws.dtf, ws.acs,
-                                          ws.status, B, L, H, chunk, false, st);
+                                          ws.status, B, L, H, chunk, st);
         });
         if (e != cudaSuccess) return cuda_status(e);
         e = timed_launch(K_STATE, st, [&] {

@@ -18,10 +18,20 @@
 // Duality and Portable O(1) Autoregressive Caching for Inference" (bqwf.cn) §1.1 says is
 // passed between chunks (the decay-weighted B^T X of each chunk).
 //
+// The kernel also forms step a1 for the items it owns (the decay factors that the state pass
+// and the scan read): dt = clip(softplus(dt_raw + dt_bias)), A = -exp(A_log), the in-block
+// cumsum acs of dt*A, stored in log2 form as colv = acs*log2(e) - log2(dt) and
+// acs2 = acs*log2(e), so that dt_s exp(acs_l - acs_s) = exp2(acs2_l - colv_s).  Source: the
+// blog walk-through's §1.1 (discretisation, chunked cumulative decay) and §1.2 (the fused
+// softplus -> clip -> exp chain); §4.1 (the decay in float32).  Tokens past L get dt = 0, so
+// their decay is 1 and their weight exactly 0 (colv = +inf).
+//
 // Structure: persistent CTAs, one per SM, each owning a contiguous range of (batch, block,
 // head) items (consecutive items share the block's B tile).  Warp-specialised:
-//   warp 0       TMA producer: B tile per (batch, block, group); x tile + the item's
-//                per-token factors into a ring of kStages stages
+//   warp 0       TMA producer: B tile per (batch, block, group); x tile per item into a ring
+//                of kStages stages
+//   warps 18..21 decay factors of an item into its stage and to global memory (warp 18 + s
+//                serves the items of stage s)
 //   warp 1       MMA issuer (one lane): 16 MMAs per item into one of two TMEM accumulators
 //   warps 2..9   transform: scale rows by w into hi (in place) and lo
 //   warps 10..17 epilogue: drain an accumulator through a swizzled shared-memory tile that
@@ -40,8 +50,9 @@ namespace ssd {
 namespace cst {
 constexpr int R = 128, P = 64, N = 128;
 constexpr int kXform = 8, kEpi = 8;
-constexpr int kThreads = (2 + kXform + kEpi) * 32;
+constexpr int kPrepWarp = 2 + kXform + kEpi;  // first of kStages decay-factor warps
 constexpr int kStages = 4;
+constexpr int kThreads = (kPrepWarp + kStages) * 32;
 constexpr uint32_t kBox = R * 128;                 // [128 rows][64 bf16], 16 KB
 constexpr uint32_t kOffB = 0;                      // B block: 2 n-boxes, 32 KB
 constexpr uint32_t kStageBytes = 2 * kBox + 1024;  // x/hi box, lo box, colv[128] + acs2[128]
@@ -55,14 +66,15 @@ constexpr uint32_t kTmemCols = 128;               // two 64-column fp32 accumula
 
 __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-    const __grid_constant__ CUtensorMap tm_s, const float *__restrict__ dtf, const float *__restrict__ acs,
-    int *__restrict__ status, int H, int G, int nk, int total) {
+    const __grid_constant__ CUtensorMap tm_s, const __nv_bfloat16 *__restrict__ dt, const float *__restrict__ A_log,
+    const float *__restrict__ dt_bias, float dt_min, float dt_max, float *__restrict__ dtf,
+    float *__restrict__ acs, int *__restrict__ status, int L, int H, int G, int nk, int total) {
     using namespace cst;
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
-    uint64_t *st_full = bars;                 // [kStages] TMA -> transform
+    uint64_t *st_full = bars;                 // [kStages] TMA + decay factors -> transform
     uint64_t *op_full = st_full + kStages;    // [kStages] transform -> MMA (operands written)
     uint64_t *st_empty = op_full + kStages;   // [kStages] MMA commit -> producer
     uint64_t *acc_full = st_empty + kStages;  // [2] MMA commit -> epilogue
@@ -74,6 +86,8 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // this call's status word starts clean (a later wait of the call may record a timeout)
+    if (blockIdx.x == 0 && tid == 0) *status = SSD_OK;
     const int first = (int)((long long)blockIdx.x * total / gridDim.x);
     const int cnt = (int)((long long)(blockIdx.x + 1) * total / gridDim.x) - first;
     if (cnt <= 0) return;
@@ -81,7 +95,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&st_full[i], 1);
+            mbar_init(&st_full[i], 2);  // the producer's expect_tx arrive + the prep warp
             mbar_init(&op_full[i], kXform);
             mbar_init(&st_empty[i], 1);
         }
@@ -133,11 +147,8 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
                 const int s = j % kStages;
                 if (j >= kStages && !wait(&st_empty[s], ((j / kStages) - 1) & 1)) break;
                 uint8_t *st = stage(j);
-                const size_t row = ((size_t)it.b * H + h) * Lp + (size_t)it.k * R;
-                mbar_arrive_expect_tx(&st_full[s], kBox + 2 * R * 4);
+                mbar_arrive_expect_tx(&st_full[s], kBox);
                 tma_load_3d(st, &tm_x, h * P, it.k * R, it.b, &st_full[s]);
-                bulk_load(st + 2 * kBox, dtf + row, R * 4, &st_full[s]);
-                bulk_load(st + 2 * kBox + R * 4, acs + row, R * 4, &st_full[s]);
             }
         }
     } else if (warp == 1) {
@@ -170,6 +181,64 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
             // every MMA (and every arrive it triggers) has landed before TMEM is released
             mma_commit(fin);
             mbar_wait(fin, 0, status);
+        }
+    } else if (warp >= kPrepWarp) {
+        // ---------------------------------------------------------------- decay factors
+        // warp kPrepWarp + s serves the items j = s, s + kStages, ... (those of stage s).  Lane
+        // i: tokens 4i .. 4i+3 of the block (the same per-lane order and warp scan as the
+        // stand-alone decay kernel, so both give the same bits).  The strided dt loads of the
+        // next item are issued before this one is processed.
+        const int s = warp - kPrepWarp;
+        auto load_raw = [&](const ItemCursor &c, float (&r)[4]) {
+            const int t0 = c.k * R + lane * 4, h = c.h();
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                r[i] = t0 + i < L ? __bfloat162float(dt[((size_t)c.b * L + t0 + i) * H + h]) : 0.f;
+        };
+        auto step = [&](ItemCursor &c) {
+#pragma unroll
+            for (int i = 0; i < kStages; ++i) c.next();
+        };
+        ItemCursor it(first + s, H, G, nk), ahead(first + s, H, G, nk);
+        float r0[4] = {0.f, 0.f, 0.f, 0.f};
+        if (s < cnt) load_raw(ahead, r0);
+        step(ahead);
+        for (int j = s; j < cnt; j += kStages) {
+            float r1[4] = {0.f, 0.f, 0.f, 0.f};
+            if (j + kStages < cnt) load_raw(ahead, r1);
+            const int h = it.h(), t0 = it.k * R + lane * 4;
+            const float bias = dt_bias ? __ldg(dt_bias + h) : 0.f;
+            const float A = -expf(__ldg(A_log + h));
+            bool ok = j < kStages || wait(&st_empty[s], ((j / kStages) - 1) & 1);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            float d[4], run = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                d[i] = t0 + i < L ? discretise_dt(r0[i], bias, dt_min, dt_max) : 0.f;
+                run += d[i] * A;
+            }
+            float acc = warp_inclusive_sum(run) - run;  // exclusive prefix of this lane
+            float cv[4], a2[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                acc += d[i] * A;
+                a2[i] = acc * kLog2e;
+                cv[i] = a2[i] - log2f(d[i]);
+            }
+            const float4 c4 = make_float4(cv[0], cv[1], cv[2], cv[3]);
+            const float4 a4 = make_float4(a2[0], a2[1], a2[2], a2[3]);
+            float *rows = reinterpret_cast<float *>(stage(j) + 2 * kBox);
+            reinterpret_cast<float4 *>(rows)[lane] = c4;
+            reinterpret_cast<float4 *>(rows + R)[lane] = a4;
+            const size_t g = ((size_t)it.b * H + h) * Lp + (size_t)t0;
+            *reinterpret_cast<float4 *>(dtf + g) = c4;
+            *reinterpret_cast<float4 *>(acs + g) = a4;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&st_full[s]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) r0[i] = r1[i];
+            step(it);
+            step(ahead);
         }
     } else if (warp < 2 + kXform) {
         // ---------------------------------------------------------------- transform
@@ -268,9 +337,10 @@ bool prefill_tc_supported(int dtype, int P, int N) {
     return dtype == SSD_DTYPE_BF16 && P == cst::P && N == cst::N;
 }
 
-cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const float *dtf, const float *acs,
-                                  float *states, int *status, int B, int L, int H, int G,
-                                  int num_sms, cudaStream_t st) {
+cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
+                                  const float *dt_bias, float dt_min, float dt_max, float *dtf, float *acs,
+                                  float *states, int *status, int B, int L, int H, int G, int num_sms,
+                                  cudaStream_t st) {
     using namespace cst;
     const int nk = cdiv(L, R);
     const int total = B * nk * H;
@@ -286,8 +356,9 @@ cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const float *dt
     if (e != cudaSuccess) return e;
     const int grid = total < num_sms ? total : num_sms;
     cudaFuncSetAttribute(chunk_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
-    chunk_state_tc_kernel<<<grid, kThreads, kSmem, st>>>(tm_x, tm_b, tm_s, dtf, acs, status, H, G, nk,
-                                                         total);
+    chunk_state_tc_kernel<<<grid, kThreads, kSmem, st>>>(tm_x, tm_b, tm_s, (const __nv_bfloat16 *)dt, A_log,
+                                                         dt_bias, dt_min, dt_max, dtf, acs, status, L, H, G,
+                                                         nk, total);
     return cudaGetLastError();
 }
 

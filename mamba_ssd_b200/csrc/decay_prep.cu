@@ -20,14 +20,9 @@
 
 namespace ssd {
 
-// Output forms: kNatural writes (dt, acs); kLog2 writes, for the tensor-core kernels,
-// (colv = acs * log2(e) - log2(dt), acs2 = acs * log2(e)), so that
-//   dt_s exp(acs_l - acs_s) = exp2(acs2_l - colv_s)
-// costs one subtraction and one ex2 per mask element (dt = 0 past the end gives colv = +inf
-// and a weight of exactly 0).
-enum DecayForm { kNatural = 0, kLog2 = 1 };
-
-template <typename T, int FORM>
+// Used by the CUDA-core path; the tensor-core path forms the same factors (in log2 form)
+// inside its block-state kernel.
+template <typename T>
 __global__ void __launch_bounds__(256) decay_prep_kernel(
     const T *__restrict__ dt, const float *__restrict__ A_log, const float *__restrict__ dt_bias,
     float dt_min, float dt_max, float *__restrict__ dtf, float *__restrict__ acs,
@@ -73,44 +68,33 @@ __global__ void __launch_bounds__(256) decay_prep_kernel(
         const size_t base = ((size_t)b * H + h) * Lp + (size_t)c * Q + lane * per;
         for (int i = 0; i < per; ++i) {
             acc += row[i] * A;
-            if (FORM == kLog2) {
-                const float a2 = acc * kLog2e;
-                acs[base + i] = a2;
-                dtf[base + i] = a2 - log2f(row[i]);
-            } else {
-                acs[base + i] = acc;
-                dtf[base + i] = row[i];
-            }
+            acs[base + i] = acc;
+            dtf[base + i] = row[i];
         }
     }
 }
 
-template <typename T, int FORM>
+template <typename T>
 static void decay_launch(dim3 grid, size_t smem, cudaStream_t st, const void *dt, const float *A_log,
                          const float *dt_bias, float dt_min, float dt_max, float *dtf, float *acs,
                          int *status, int L, int H, int chunk, int nc) {
-    cudaFuncSetAttribute(decay_prep_kernel<T, FORM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    decay_prep_kernel<T, FORM><<<grid, 256, smem, st>>>((const T *)dt, A_log, dt_bias, dt_min, dt_max, dtf,
-                                                        acs, status, L, H, chunk, nc);
+    cudaFuncSetAttribute(decay_prep_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    decay_prep_kernel<T><<<grid, 256, smem, st>>>((const T *)dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, status,
+                                                  L, H, chunk, nc);
 }
 
 cudaError_t launch_decay_prep(int dtype, const void *dt, const float *A_log, const float *dt_bias,
                               float dt_min, float dt_max, float *dtf, float *acs, int *status, int B,
-                              int L, int H, int chunk, bool log2_form, cudaStream_t st) {
+                              int L, int H, int chunk, cudaStream_t st) {
     const int nc = cdiv(L, chunk);
     dim3 grid(nc, B, cdiv(H, 8));
     const size_t smem = sizeof(float) * 8 * (chunk + 1);
-    if (dtype == SSD_DTYPE_BF16) {
-        if (log2_form)
-            decay_launch<__nv_bfloat16, kLog2>(grid, smem, st, dt, A_log, dt_bias, dt_min, dt_max, dtf, acs,
-                                               status, L, H, chunk, nc);
-        else
-            decay_launch<__nv_bfloat16, kNatural>(grid, smem, st, dt, A_log, dt_bias, dt_min, dt_max, dtf, acs,
-                                                  status, L, H, chunk, nc);
-    } else {
-        decay_launch<float, kNatural>(grid, smem, st, dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, status, L,
-                                      H, chunk, nc);
-    }
+    if (dtype == SSD_DTYPE_BF16)
+        decay_launch<__nv_bfloat16>(grid, smem, st, dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, status, L, H,
+                                    chunk, nc);
+    else
+        decay_launch<float>(grid, smem, st, dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, status, L, H, chunk,
+                            nc);
     return cudaGetLastError();
 }
 

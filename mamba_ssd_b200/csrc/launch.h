@@ -14,7 +14,8 @@ namespace ssd {
 //   acs    [B][H][Lp]          inclusive cumsum of dt*A inside each block; on the tensor-core
 //                              path acs2 = that cumsum times log2(e)
 //   states [B][nb][H][P][N]    fp32 block states; the CUDA-core path overwrites them in
-//                              place with the state each block starts from (h_prev)
+//                              place with the state each block starts from (h_prev); the
+//                              tensor-core path stores each transposed, [N][P]
 //   hT     [B][nb][H][N][P]    (tensor-core path) h_prev of each block, bf16, transposed
 // with nb = ceil(L / block), Lp = nb * block.  The block is the caller's chunk on the
 // CUDA-core path and 128 tokens (the tcgen05 M) on the tensor-core path.
@@ -29,18 +30,20 @@ size_t prefill_workspace_bytes(int B, int L, int H, int P, int N, int block, boo
 PrefillWorkspace carve_prefill_workspace(void *base, int B, int L, int H, int P, int N, int block,
                                          bool transposed_bf16);
 
-// log2_form: write colv = acs*log2(e) - log2(dt) and acs2 = acs*log2(e) (tensor-core path)
-// instead of dt and acs.
+// Step a1 for the CUDA-core path: writes dt and acs (natural form) and resets the status word.
 cudaError_t launch_decay_prep(int dtype, const void *dt, const float *A_log, const float *dt_bias,
                               float dt_min, float dt_max, float *dtf, float *acs, int *status, int B,
-                              int L, int H, int chunk, bool log2_form, cudaStream_t st);
+                              int L, int H, int chunk, cudaStream_t st);
 
 // tensor-core prefill (bf16 storage, P = 64, N = 128), 128-token blocks
 constexpr int kTcBlock = 128;
 bool prefill_tc_supported(int dtype, int P, int N);
-cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const float *dtf, const float *acs,
-                                  float *states, int *status, int B, int L, int H, int G,
-                                  int num_sms, cudaStream_t st);
+// chunk_state_tc also forms the log2-form decay factors (dtf = colv, acs = acs2) from dt and
+// resets the status word: it is the first kernel of a tensor-core prefill call.
+cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
+                                  const float *dt_bias, float dt_min, float dt_max, float *dtf, float *acs,
+                                  float *states, int *status, int B, int L, int H, int G, int num_sms,
+                                  cudaStream_t st);
 
 cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, const float *dtf,
                                  const float *acs, const __nv_bfloat16 *hT, const float *D, void *y,
