@@ -67,6 +67,19 @@ inline int cuda_status(cudaError_t e) {
     return SSD_ERR_CUDA;
 }
 
+}  // namespace
+
+namespace ssd {
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char *v = getenv("SSD_PDL");
+        return !(v && v[0] == '0');
+    }();
+    return on;
+}
+}  // namespace ssd
+
+namespace {
 // Tensor-core kernels are used wherever they apply, unless SSD_PREFILL_KERNELS=simt is set in
 // the environment (then every shape runs on the float32 CUDA-core kernels).
 bool use_tensor_cores() {

@@ -128,6 +128,8 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // prologue done: from here on global memory is touched, after the previous kernel
+    grid_dependency_wait();
 
     auto stage = [&](int j) { return smem + kOffStage + (uint32_t)(j % kStages) * kStageBytes; };
     // a bounded wait that gives up at once when another role has already timed out
@@ -362,6 +364,7 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
         while (globaltimer() - t0 < 2000000ull) {
         }
     }
+    allow_dependents();  // this CTA's work is done: the next kernel may take its SM
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_free(tmem, kTmemCols);
@@ -390,9 +393,8 @@ cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, 
     if (e != cudaSuccess) return e;
     const int grid = total < num_sms ? total : num_sms;
     cudaFuncSetAttribute(chunk_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
-    chunk_scan_tc_kernel<<<grid, kThreads, kSmem, st>>>(tm_x, tm_b, tm_c, tm_h, tm_y, dtf, acs, D, status, H, G,
-                                                        nk, total);
-    return cudaGetLastError();
+    return launch_pdl(chunk_scan_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, tm_x, tm_b, tm_c, tm_h, tm_y,
+                      dtf, acs, D, status, H, G, nk, total);
 }
 
 }  // namespace ssd

@@ -86,8 +86,6 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // this call's status word starts clean (a later wait of the call may record a timeout)
-    if (blockIdx.x == 0 && tid == 0) *status = SSD_OK;
     const int first = (int)((long long)blockIdx.x * total / gridDim.x);
     const int cnt = (int)((long long)(blockIdx.x + 1) * total / gridDim.x) - first;
     if (cnt <= 0) return;
@@ -117,6 +115,10 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // prologue done: from here on global memory is touched, after the previous kernel
+    grid_dependency_wait();
+    // this call's status word starts clean (a later wait of the call may record a timeout)
+    if (blockIdx.x == 0 && tid == 0) *status = SSD_OK;
 
     auto stage = [&](int j) { return smem + kOffStage + (uint32_t)(j % kStages) * kStageBytes; };
     // a bounded wait that gives up at once when another role has already timed out
@@ -328,6 +330,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
         while (globaltimer() - t0 < 2000000ull) {
         }
     }
+    allow_dependents();  // this CTA's work is done: the next kernel may take its SM
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_free(tmem, kTmemCols);
@@ -356,10 +359,9 @@ cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const void *dt,
     if (e != cudaSuccess) return e;
     const int grid = total < num_sms ? total : num_sms;
     cudaFuncSetAttribute(chunk_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
-    chunk_state_tc_kernel<<<grid, kThreads, kSmem, st>>>(tm_x, tm_b, tm_s, (const __nv_bfloat16 *)dt, A_log,
-                                                         dt_bias, dt_min, dt_max, dtf, acs, status, L, H, G,
-                                                         nk, total);
-    return cudaGetLastError();
+    return launch_pdl(chunk_state_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, tm_x, tm_b, tm_s,
+                      (const __nv_bfloat16 *)dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, status, L, H, G, nk,
+                      total);
 }
 
 }  // namespace ssd

@@ -54,6 +54,15 @@ __device__ __forceinline__ float warp_inclusive_sum(float v) {
     return v;
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization
+// may start while the kernel before it in the stream is still running; grid_dependency_wait()
+// blocks the calling thread until that kernel has completed and its memory operations are
+// visible (a no-op for an ordinary launch), so every global access comes after it.
+// allow_dependents() lets the next such kernel be scheduled once every CTA of this grid has
+// called it (or exited).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __host__ __device__ constexpr inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ constexpr inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 

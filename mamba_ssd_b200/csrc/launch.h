@@ -7,6 +7,26 @@
 
 namespace ssd {
 
+// Launches of the tensor-core prefill kernels use programmatic stream serialization (each may
+// be scheduled while the kernel before it finishes; the kernels order every global access
+// after griddepcontrol.wait).  SSD_PDL=0 in the environment turns it off.
+bool pdl_enabled();
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Prefill workspace layout, 256-byte aligned pieces:
 //   status int32 (256-byte slot): SSD_OK, or SSD_ERR_TIMEOUT if a bounded wait gave up
 //   dtf    [B][H][Lp]          clipped dt per token (0 past the end of the sequence); on the

@@ -71,6 +71,7 @@ __global__ void __launch_bounds__(256) state_pass_t_kernel(const float *__restri
                                                            __nv_bfloat16 *__restrict__ hT, int H,
                                                            int P, int N, int nc, int Q) {
     constexpr int kAhead = 8;
+    grid_dependency_wait();  // the block states come from the kernel before
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     const int p0 = (t * 4) % P, n = (t * 4) / P;
     const int h = blockIdx.y, b = blockIdx.z;
@@ -111,6 +112,7 @@ __global__ void __launch_bounds__(256) state_pass_t_kernel(const float *__restri
 #pragma unroll
         for (int i = 0; i < 4; ++i) h_final[bh * PN + (size_t)(p0 + i) * N + n] = s[i];
     }
+    allow_dependents();
 }
 
 cudaError_t launch_state_pass_t(const float *states, const float *acs, const float *h0, float *h_final,
@@ -118,8 +120,8 @@ cudaError_t launch_state_pass_t(const float *states, const float *acs, const flo
                                 cudaStream_t st) {
     const int nc = cdiv(L, chunk);
     dim3 grid(cdiv(P * N / 4, 256), H, B);
-    state_pass_t_kernel<<<grid, 256, 0, st>>>(states, acs, h0, h_final, hT, H, P, N, nc, chunk);
-    return cudaGetLastError();
+    return launch_pdl(state_pass_t_kernel, grid, dim3(256), 0, st, states, acs, h0, h_final, hT, H, P, N, nc,
+                      chunk);
 }
 
 cudaError_t launch_state_pass(float *states, const float *acs, const float *h0, float *h_final,
