@@ -153,11 +153,19 @@ SSD_API int ssd_chunk_scan_fwd_noalloc(const void *x, const void *dt, const floa
 
 /*
  * Bytes of device workspace that ssd_decode_step needs (a multiple of 256).  The
- * workspace holds one arrival counter per (batch, group): it must be zero-filled once
- * before its first use, and every completed call leaves it zero-filled again, so one
- * zeroed workspace serves any number of consecutive calls on one stream.
+ * workspace holds a status word and one arrival counter per (batch, group): it must be
+ * zero-filled once before its first use, and every completed call leaves it zero-filled
+ * again, so one zeroed workspace serves any number of consecutive calls on one stream.
  */
 SSD_API size_t ssd_decode_workspace_size(int B, int G);
+
+/*
+ * Diagnostic: synchronises `stream` and returns the status word the last ssd_decode_step
+ * on `workspace` left; SSD_ERR_INVALID_ARG for a NULL workspace, SSD_ERR_CUDA if the stream
+ * reported an error.  The decode kernel has no waits and always leaves SSD_OK; the word is
+ * there so that a kernel with bounded waits can report SSD_ERR_TIMEOUT without an ABI change.
+ */
+SSD_API int ssd_decode_status(const void *workspace, void *stream);
 
 /*
  * One cached decode step for one layer ([blog §2.1, §2.2]):

@@ -115,12 +115,25 @@ def ssd_chunk_scan_fwd_noalloc(x, dt, A_log, Bm, Cm, D=None, chunk=256, h0=None,
     return y, h_final
 
 
+def ssd_chunk_scan_status(workspace, stream=None):
+    """Synchronises the stream and returns the status word the last prefill on `workspace`
+    left: SSD_OK (0), or SSD_ERR_TIMEOUT (5) if a bounded wait in a kernel gave up."""
+    return _lib.lib().ssd_chunk_scan_status(_ptr(workspace), _stream(stream))
+
+
+def ssd_decode_status(workspace, stream=None):
+    """Synchronises the stream and returns the status word the last decode step on
+    `workspace` left: SSD_OK (0), or SSD_ERR_TIMEOUT (5)."""
+    return _lib.lib().ssd_decode_status(_ptr(workspace), _stream(stream))
+
+
 def ssd_decode_workspace_size(B, G):
     return int(_lib.lib().ssd_decode_workspace_size(B, G))
 
 
 def decode_workspace(B, G, device="cuda"):
-    """A zero-filled decode workspace (arrival counters), reusable across calls."""
+    """A zero-filled decode workspace (status word and arrival counters), reusable across
+    calls on one stream."""
     return torch.zeros(max(ssd_decode_workspace_size(B, G), 256), device=device, dtype=torch.uint8)
 
 

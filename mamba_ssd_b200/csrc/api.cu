@@ -267,9 +267,20 @@ int ssd_chunk_scan_status(const void *workspace, void *stream) {
     return v;
 }
 
+// Decode workspace: a status word (256-byte slot), then one arrival counter per (batch, group).
 size_t ssd_decode_workspace_size(int B, int G) {
     if (B <= 0 || G <= 0) return 0;
-    return ssd::align_up(sizeof(unsigned) * (size_t)B * G, 256);
+    return 256 + ssd::align_up(sizeof(unsigned) * (size_t)B * G, 256);
+}
+
+int ssd_decode_status(const void *workspace, void *stream) {
+    if (!workspace) return SSD_ERR_INVALID_ARG;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(e);
+    int v = 0;
+    e = cudaMemcpy(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e);
+    return v;
 }
 
 int ssd_decode_step(float *ssm_state, void *conv_state, const void *xBC_t, const void *dt_t,
@@ -298,7 +309,8 @@ int ssd_decode_step(float *ssm_state, void *conv_state, const void *xBC_t, const
     cudaError_t e = timed_launch(K_DECODE, st, [&] {
         return ssd::launch_decode_step(dtype, ssm_state, conv_state, xBC_t, dt_t, A_log, D, dt_bias,
                                        dt_min, dt_max, conv_w, conv_b, y_t, B, H, P, G, N, K,
-                                       static_cast<unsigned *>(workspace), st);
+                                       static_cast<int *>(workspace),
+                                       reinterpret_cast<unsigned *>(static_cast<char *>(workspace) + 256), st);
     });
     return cuda_status(e);
 }

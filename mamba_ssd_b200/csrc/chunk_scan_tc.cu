@@ -240,6 +240,7 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
         int tiles = 0;
         for (int j = 0; j < cnt; ++j, it.next()) {
             const int s = j % kStages, t = j & 1;
+            const float d = D ? __ldg(D + it.h()) : 0.f;  // issued before the waits
             if (j == 0 || it.tile_first()) {
                 if (!__all_sync(0xffffffffu, wait(cb_full, tiles & 1))) break;
                 ++tiles;
@@ -252,7 +253,6 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
             const float *colv = reinterpret_cast<const float *>(stage(j) + kStRows);
             const float *acs2 = colv + R;
             const float al = acs2[myrow];
-            const float d = D ? __ldg(D + it.h()) : 0.f;
             const uint32_t set = tmem + lane_base + kSet0 + t * kSet;
 #pragma unroll
             for (int bi = 0; bi < 2; ++bi) {

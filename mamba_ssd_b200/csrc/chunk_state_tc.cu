@@ -201,16 +201,26 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
 #pragma unroll
             for (int i = 0; i < kStages; ++i) c.next();
         };
+        auto load_par = [&](const ItemCursor &c, float &bias, float &alog) {
+            bias = dt_bias ? __ldg(dt_bias + c.h()) : 0.f;
+            alog = __ldg(A_log + c.h());
+        };
         ItemCursor it(first + s, H, G, nk), ahead(first + s, H, G, nk);
-        float r0[4] = {0.f, 0.f, 0.f, 0.f};
-        if (s < cnt) load_raw(ahead, r0);
+        float r0[4] = {0.f, 0.f, 0.f, 0.f}, b0 = 0.f, l0 = 0.f;
+        if (s < cnt) {
+            load_raw(ahead, r0);
+            load_par(ahead, b0, l0);
+        }
         step(ahead);
         for (int j = s; j < cnt; j += kStages) {
-            float r1[4] = {0.f, 0.f, 0.f, 0.f};
-            if (j + kStages < cnt) load_raw(ahead, r1);
+            float r1[4] = {0.f, 0.f, 0.f, 0.f}, b1 = 0.f, l1 = 0.f;
+            if (j + kStages < cnt) {
+                load_raw(ahead, r1);
+                load_par(ahead, b1, l1);
+            }
             const int h = it.h(), t0 = it.k * R + lane * 4;
-            const float bias = dt_bias ? __ldg(dt_bias + h) : 0.f;
-            const float A = -expf(__ldg(A_log + h));
+            const float bias = b0;
+            const float A = -expf(l0);
             bool ok = j < kStages || wait(&st_empty[s], ((j / kStages) - 1) & 1);
             if (!__all_sync(0xffffffffu, ok)) break;
             float d[4], run = 0.f;
@@ -239,6 +249,8 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
             if (lane == 0) mbar_arrive(&st_full[s]);
 #pragma unroll
             for (int i = 0; i < 4; ++i) r0[i] = r1[i];
+            b0 = b1;
+            l0 = l1;
             step(it);
             step(ahead);
         }

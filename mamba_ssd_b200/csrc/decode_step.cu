@@ -23,8 +23,11 @@
 // x-channels (it is their only reader and writer) and all 2N B/C channels of its group,
 // which every CTA of the group needs.  Those B/C conv-cache entries may only be rolled
 // after every CTA of the group has read them: each CTA bumps a per-(batch, group) arrival
-// counter once its reads are done, and the CTA that arrives last rolls the B/C cache and
-// resets the counter to zero (no CTA ever waits, so nothing can hang).
+// counter as soon as its reads are done -- from a thread that has issued no global store, so
+// its fence costs nothing and the atomic overlaps the state update -- and the CTA that arrives
+// last rolls the B/C cache at its end and resets the counter to zero (no CTA ever waits, so
+// nothing can hang).  The kernel has no bounded waits: it resets the workspace status word to
+// SSD_OK and never sets it otherwise.
 #include "common.cuh"
 #include "launch.h"
 
@@ -37,7 +40,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
     float *__restrict__ ssm, T *__restrict__ conv_state, const T *__restrict__ xBC_t,
     const T *__restrict__ dt_t, const float *__restrict__ A_log, const float *__restrict__ D,
     const float *__restrict__ dt_bias, float dt_min, float dt_max, const T *__restrict__ conv_w,
-    const T *__restrict__ conv_b, T *__restrict__ y_t, int H, int P, int G,
+    const T *__restrict__ conv_b, T *__restrict__ y_t, int H, int P, int G, int *__restrict__ status,
     unsigned *__restrict__ counters) {
     constexpr int V = (N > 128) ? N / 128 : 1;  // float4 per thread per row
     constexpr int TPR = N / (4 * V);            // threads per row (<= 32, power of two)
@@ -57,6 +60,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
     const int Cc = HP + 2 * GN;
     const int tid = threadIdx.x;
     const int r_in_pass = tid / TPR, lane_in_row = tid % TPR;
+    constexpr int kArriver = kDecThreads - 1;  // no x channel (ROWS < kDecThreads): no store before the arrival
+    static_assert(ROWS < kDecThreads, "the arriving thread must not own an x channel");
+
+    grid_dependency_wait();  // every global access comes after the kernel before
+    if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *status = SSD_OK;
 
     // ---- issue every independent load first ----
     float4 st[PASSES][V];
@@ -135,6 +143,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
     }
     __syncthreads();  // conv outputs and dt are in shared memory; B/C cache reads are done
 
+    // ---- arrival: the CTA that arrives last for its (batch, group) rolls the B/C cache below ----
+    if (tid == kArriver) {
+        __threadfence();
+        const unsigned ctas = (unsigned)((H / G) * P / ROWS);
+        const unsigned prev = atomicAdd(&counters[b * G + g], 1u);
+        s_last = (prev == ctas - 1);
+    }
+
     // ---- state update and output ----
     const float dt = s_dt, a = s_a, dsk = s_d;
 #pragma unroll
@@ -165,16 +181,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
         if (r < ROWS && lane_in_row == 0) y_t[(size_t)b * HP + row0 + r] = from_f<T>(part + dsk * xv);
     }
 
-    // ---- arrival: the last CTA of the (batch, group) rolls the shared B/C conv cache ----
-    // (every read of that cache by this CTA happened before the __syncthreads above)
-
-    if (tid == 0) {
-        __threadfence();
-        const unsigned ctas = (unsigned)((H / G) * P / ROWS);
-        const unsigned prev = atomicAdd(&counters[b * G + g], 1u);
-        s_last = (prev == ctas - 1);
-    }
-    __syncthreads();
+    __syncthreads();  // s_last is visible
     if (s_last) {
         // every CTA of this (batch, group) has read the B/C cache: roll it
         __threadfence();
@@ -190,41 +197,41 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
         }
         if (tid == 0) atomicExch(&counters[b * G + g], 0u);
     }
+    allow_dependents();
 }
 
 template <typename T, int N, int K, int ROWS>
 static cudaError_t decode_launch(float *ssm, void *conv_state, const void *xBC_t, const void *dt_t,
                                  const float *A_log, const float *D, const float *dt_bias, float dt_min,
                                  float dt_max, const void *conv_w, const void *conv_b, void *y_t,
-                                 int B, int H, int P, int G, unsigned *counters, cudaStream_t st) {
+                                 int B, int H, int P, int G, int *status, unsigned *counters, cudaStream_t st) {
     dim3 grid(H * P / ROWS, B);
-    decode_step_kernel<T, N, K, ROWS><<<grid, kDecThreads, 0, st>>>(
-        ssm, (T *)conv_state, (const T *)xBC_t, (const T *)dt_t, A_log, D, dt_bias, dt_min, dt_max,
-        (const T *)conv_w, (const T *)conv_b, (T *)y_t, H, P, G, counters);
-    return cudaGetLastError();
+    return launch_pdl(decode_step_kernel<T, N, K, ROWS>, grid, dim3(kDecThreads), 0, st, ssm, (T *)conv_state,
+                      (const T *)xBC_t, (const T *)dt_t, A_log, D, dt_bias, dt_min, dt_max, (const T *)conv_w,
+                      (const T *)conv_b, (T *)y_t, H, P, G, status, counters);
 }
 
 template <typename T, int N, int K>
 static cudaError_t decode_rows(bool wide, float *ssm, void *conv_state, const void *xBC_t, const void *dt_t,
                                const float *A_log, const float *D, const float *dt_bias, float dt_min,
                                float dt_max, const void *conv_w, const void *conv_b, void *y_t, int B,
-                               int H, int P, int G, unsigned *counters, cudaStream_t st) {
+                               int H, int P, int G, int *status, unsigned *counters, cudaStream_t st) {
     if (wide)
         return decode_launch<T, N, K, 64>(ssm, conv_state, xBC_t, dt_t, A_log, D, dt_bias, dt_min, dt_max,
-                                          conv_w, conv_b, y_t, B, H, P, G, counters, st);
+                                          conv_w, conv_b, y_t, B, H, P, G, status, counters, st);
     return decode_launch<T, N, K, 16>(ssm, conv_state, xBC_t, dt_t, A_log, D, dt_bias, dt_min, dt_max,
-                                      conv_w, conv_b, y_t, B, H, P, G, counters, st);
+                                      conv_w, conv_b, y_t, B, H, P, G, status, counters, st);
 }
 
 template <typename T, int N>
 static cudaError_t decode_k(int K, bool wide, float *ssm, void *conv_state, const void *xBC_t,
                             const void *dt_t, const float *A_log, const float *D, const float *dt_bias,
                             float dt_min, float dt_max, const void *conv_w, const void *conv_b, void *y_t,
-                            int B, int H, int P, int G, unsigned *counters, cudaStream_t st) {
+                            int B, int H, int P, int G, int *status, unsigned *counters, cudaStream_t st) {
 #define SSD_DK(KK)                                                                                   \
     case KK:                                                                                         \
         return decode_rows<T, N, KK>(wide, ssm, conv_state, xBC_t, dt_t, A_log, D, dt_bias, dt_min, \
-                                     dt_max, conv_w, conv_b, y_t, B, H, P, G, counters, st);
+                                     dt_max, conv_w, conv_b, y_t, B, H, P, G, status, counters, st);
     switch (K) {
         SSD_DK(2) SSD_DK(3) SSD_DK(4) SSD_DK(5) SSD_DK(6) SSD_DK(7) SSD_DK(8)
     }
@@ -236,13 +243,14 @@ cudaError_t launch_decode_step(int dtype, float *ssm_state, void *conv_state, co
                                const void *dt_t, const float *A_log, const float *D,
                                const float *dt_bias, float dt_min, float dt_max,
                                const void *conv_w, const void *conv_b, void *y_t, int B, int H,
-                               int P, int G, int N, int K, unsigned *counters, cudaStream_t st) {
+                               int P, int G, int N, int K, int *status, unsigned *counters,
+                               cudaStream_t st) {
     // 64 rows per CTA once the batch gives enough CTAs; 16 otherwise
     const bool wide = (P % 64 == 0) && (B >= 4);
 #define SSD_DN(T, NN)                                                                              \
     case NN:                                                                                       \
         return decode_k<T, NN>(K, wide, ssm_state, conv_state, xBC_t, dt_t, A_log, D, dt_bias,      \
-                               dt_min, dt_max, conv_w, conv_b, y_t, B, H, P, G, counters, st);
+                               dt_min, dt_max, conv_w, conv_b, y_t, B, H, P, G, status, counters, st);
     if (dtype == SSD_DTYPE_BF16) {
         switch (N) { SSD_DN(__nv_bfloat16, 16) SSD_DN(__nv_bfloat16, 32) SSD_DN(__nv_bfloat16, 64)
                      SSD_DN(__nv_bfloat16, 128) SSD_DN(__nv_bfloat16, 256) }

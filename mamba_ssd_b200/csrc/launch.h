@@ -88,7 +88,8 @@ cudaError_t launch_decode_step(int dtype, float *ssm_state, void *conv_state, co
                                const void *dt_t, const float *A_log, const float *D,
                                const float *dt_bias, float dt_min, float dt_max,
                                const void *conv_w, const void *conv_b, void *y_t, int B, int H,
-                               int P, int G, int N, int K, unsigned *counters, cudaStream_t st);
+                               int P, int G, int N, int K, int *status, unsigned *counters,
+                               cudaStream_t st);
 
 cudaError_t launch_causal_conv1d(int dtype, const void *xBC, const void *conv_w,
                                  const void *conv_b, void *out, void *conv_state_out, int B,

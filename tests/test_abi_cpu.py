@@ -120,8 +120,11 @@ def test_decode_validation(kw, want):
 
 
 def test_decode_workspace_size():
-    assert L.ssd_decode_workspace_size(1, 1) == 256
-    assert L.ssd_decode_workspace_size(16, 8) == 512
+    # a 256-byte status slot, then one 4-byte counter per (batch, group) rounded up to 256
+    assert L.ssd_decode_workspace_size(1, 1) == 512
+    assert L.ssd_decode_workspace_size(16, 8) == 768
+    assert L.ssd_decode_workspace_size(64, 2) == 768
+    assert L.ssd_decode_workspace_size(65, 2) == 1024
     assert L.ssd_decode_workspace_size(0, 1) == 0
 
 
