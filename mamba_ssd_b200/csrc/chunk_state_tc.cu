@@ -11,8 +11,10 @@
 // MN-major straight from 128-byte-swizzled tiles.  The fp32 block state feeds the float32
 // state pass and finally h_final, whose tolerance (1e-3 relative to its RMS) is tighter than
 // one bf16 rounding of w_s x_s (RMS relative error 2^-9/sqrt(3) = 1.1e-3).  So X'' is split
-// into bf16 hi + lo parts (hi = bf16(v), lo = bf16(v - hi), |v - hi - lo| <= 2^-17 |v|) and
-// both are accumulated into the same fp32 TMEM accumulator: 2 x 8 MMAs of K=16.
+// into bf16 hi + lo parts (hi = bf16(v), lo = bf16(v - hi), |v - hi - lo| <= 2^-17 |v|).  The lo
+// box sits one MN atom after the hi box, so [hi | lo] is a single N = 128 operand: 8 MMAs of
+// K=16 (M128 N128) into a 128-column fp32 accumulator whose halves the epilogue adds -- each
+// MMA reads the shared A operand once for both parts.
 //
 // Source: the per-chunk state that the blog walk-through of "Compiler-First State Space
 // Duality and Portable O(1) Autoregressive Caching for Inference" (bqwf.cn) §1.1 says is
@@ -32,7 +34,7 @@
 //                of kStages stages
 //   warps 18..21 decay factors of an item into its stage and to global memory (warp 18 + s
 //                serves the items of stage s)
-//   warp 1       MMA issuer (one lane): 16 MMAs per item into one of two TMEM accumulators
+//   warp 1       MMA issuer (one lane): 8 MMAs per item into one of two TMEM accumulators
 //   warps 2..9   transform: scale rows by w into hi (in place) and lo
 //   warps 10..17 epilogue: drain an accumulator through a swizzled shared-memory tile that
 //                one TMA store per 32-column half writes out (S^T, [N][P], fp32)
@@ -61,7 +63,7 @@ constexpr uint32_t kOffOut = kOffStage + kStages * kStageBytes;  // S^T staging:
 constexpr uint32_t kOffBar = kOffOut + 2 * kBox;
 constexpr int kEpiBar = 1;  // named barrier of the epilogue warps
 constexpr uint32_t kSmem = kOffBar + 256 + 1024;  // + slack for 1024-byte alignment
-constexpr uint32_t kTmemCols = 128;               // two 64-column fp32 accumulators
+constexpr uint32_t kTmemCols = 256;               // two 128-column fp32 accumulators [hi | lo]
 }  // namespace cst
 
 __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
@@ -156,7 +158,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(128, 64, true, true);
+            constexpr uint32_t idesc = idesc_bf16_f32(128, 128, true, true);  // N = [hi | lo]
             const uint64_t da = desc_mnmajor_sw128(smem_u32(smem + kOffB), kBox);
             ItemCursor it(first, H, G, nk);
             int tiles = 0;
@@ -169,13 +171,11 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
                 if (!wait(&op_full[s], (j / kStages) & 1)) break;
                 if (j >= 2 && !wait(&acc_empty[a], ((j >> 1) - 1) & 1)) break;
                 tc_fence_after();
-                const uint64_t dh = desc_mnmajor_sw128(smem_u32(stage(j)), kBox), dl = desc_add(dh, kBox);
-                const uint32_t d = tmem + (uint32_t)(a * 64);
+                const uint64_t dh = desc_mnmajor_sw128(smem_u32(stage(j)), kBox);  // [hi | lo] at LBO kBox
+                const uint32_t d = tmem + (uint32_t)(a * 128);
 #pragma unroll
                 for (int kk = 0; kk < R / 16; ++kk)
                     mma_ss(d, desc_add(da, kk * 2048), desc_add(dh, kk * 2048), idesc, kk > 0 ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < R / 16; ++kk) mma_ss(d, desc_add(da, kk * 2048), desc_add(dl, kk * 2048), idesc, 1u);
                 mma_commit(&acc_full[a]);
                 mma_commit(&st_empty[s]);
                 if (j == cnt - 1 || it.tile_last()) mma_commit(b_empty);
@@ -308,10 +308,16 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
             float v[32];
             if (ok) {
                 tc_fence_after();
-                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 64 + half * 32);
+                // columns [0, 64) hold the hi part's products, [64, 128) the lo part's
+                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 128 + half * 32);
+                float w[32];
                 tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(&v[0]));
                 tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+                tmem_ld16(taddr + 64, *reinterpret_cast<float(*)[16]>(&w[0]));
+                tmem_ld16(taddr + 80, *reinterpret_cast<float(*)[16]>(&w[16]));
                 tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] += w[i];
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[a]);
