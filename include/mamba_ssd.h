@@ -206,6 +206,17 @@ SSD_API int ssd_causal_conv1d_fwd(const void *xBC, const void *conv_w, const voi
                           void *stream);
 
 /*
+ * Self-test of the bounded waits (no counterpart in the pages; the failure path of the
+ * tensor-core kernels).  Launches one warp that waits, with the same bounded-wait code the
+ * prefill kernels use, on an mbarrier that no thread ever arrives at, giving up after
+ * `limit_us` microseconds (1 .. 1000000).  It then stores SSD_ERR_TIMEOUT into `status` (one
+ * device int, caller-owned) and returns; nothing faults or hangs and the context stays
+ * usable.  Returns SSD_ERR_INVALID_ARG for a NULL or misaligned status or a limit out of
+ * range, SSD_ERR_CUDA if the launch failed, else SSD_OK (asynchronous on `stream`).
+ */
+SSD_API int ssd_selftest_wait_timeout(int *status, int limit_us, void *stream);
+
+/*
  * Profiling hooks (host-side bookkeeping; no device memory is allocated).
  *
  * ssd_kernel_launch_count: kernels this library has enqueued in this process so far

@@ -127,6 +127,15 @@ def ssd_decode_status(workspace, stream=None):
     return _lib.lib().ssd_decode_status(_ptr(workspace), _stream(stream))
 
 
+def ssd_selftest_wait_timeout(limit_us, device="cuda", stream=None):
+    """Runs the bounded-wait self-test (a wait on an mbarrier that nothing arrives at, given
+    up after `limit_us` microseconds) and returns the status it recorded: SSD_ERR_TIMEOUT."""
+    status = torch.zeros(1, device=device, dtype=torch.int32)
+    check(_lib.lib().ssd_selftest_wait_timeout(_ptr(status), int(limit_us), _stream(stream)),
+          "ssd_selftest_wait_timeout")
+    return int(status.item())
+
+
 def ssd_decode_workspace_size(B, G):
     return int(_lib.lib().ssd_decode_workspace_size(B, G))
 

@@ -338,6 +338,12 @@ int ssd_causal_conv1d_fwd(const void *xBC, const void *conv_w, const void *conv_
     }));
 }
 
+int ssd_selftest_wait_timeout(int *status, int limit_us, void *stream) {
+    if (!status || (reinterpret_cast<uintptr_t>(status) & 3u) || limit_us < 1 || limit_us > 1000000)
+        return SSD_ERR_INVALID_ARG;
+    return cuda_status(ssd::launch_selftest_wait(status, limit_us, static_cast<cudaStream_t>(stream)));
+}
+
 long long ssd_kernel_launch_count(void) { return g_launches.load(); }
 
 int ssd_kernel_timer_enable(int on) {

@@ -33,10 +33,10 @@
 
 namespace ssd {
 
-constexpr int kDecThreads = 128;
-
-template <typename T, int N, int K, int ROWS>
-__global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
+// THREADS = 128 with 16 rows per CTA (small batches: more CTAs), 256 with 64 rows: 8 float4 of
+// state per thread (64 registers), four CTAs to an SM.
+template <typename T, int N, int K, int ROWS, int THREADS>
+__global__ void __launch_bounds__(THREADS) decode_step_kernel(
     float *__restrict__ ssm, T *__restrict__ conv_state, const T *__restrict__ xBC_t,
     const T *__restrict__ dt_t, const float *__restrict__ A_log, const float *__restrict__ D,
     const float *__restrict__ dt_bias, float dt_min, float dt_max, const T *__restrict__ conv_w,
@@ -44,9 +44,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
     unsigned *__restrict__ counters) {
     constexpr int V = (N > 128) ? N / 128 : 1;  // float4 per thread per row
     constexpr int TPR = N / (4 * V);            // threads per row (<= 32, power of two)
-    constexpr int RPP = kDecThreads / TPR;      // rows per pass
+    constexpr int RPP = THREADS / TPR;      // rows per pass
     constexpr int PASSES = (ROWS + RPP - 1) / RPP;
-    constexpr int BC_PER = (2 * N + kDecThreads - 1) / kDecThreads;  // B/C channels per thread
+    constexpr int BC_PER = (2 * N + THREADS - 1) / THREADS;  // B/C channels per thread
 
     __shared__ float uB[N], uC[N], ux[ROWS];
     __shared__ float s_dt, s_a, s_d;
@@ -60,8 +60,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
     const int Cc = HP + 2 * GN;
     const int tid = threadIdx.x;
     const int r_in_pass = tid / TPR, lane_in_row = tid % TPR;
-    constexpr int kArriver = kDecThreads - 1;  // no x channel (ROWS < kDecThreads): no store before the arrival
-    static_assert(ROWS < kDecThreads, "the arriving thread must not own an x channel");
+    constexpr int kArriver = THREADS - 1;  // no x channel (ROWS < THREADS): no store before the arrival
+    static_assert(ROWS < THREADS, "the arriving thread must not own an x channel");
 
     grid_dependency_wait();  // every global access comes after the kernel before
     if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *status = SSD_OK;
@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
     float bc_win[BC_PER][K], bc_w[BC_PER][K], bc_bias[BC_PER];
 #pragma unroll
     for (int q = 0; q < BC_PER; ++q) {
-        const int i = tid + q * kDecThreads;
+        const int i = tid + q * THREADS;
         if (i < 2 * N) {
             const int cc = HP + (i < N ? g * N + i : GN + g * N + (i - N));
             const T *cs = conv_state + ((size_t)b * Cc + cc) * (K - 1);
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
     // ---- conv outputs, x-channel cache roll, discretisation ----
 #pragma unroll
     for (int q = 0; q < BC_PER; ++q) {
-        const int i = tid + q * kDecThreads;
+        const int i = tid + q * THREADS;
         if (i < 2 * N) {
             float acc = bc_bias[q];
 #pragma unroll
@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
         __threadfence();
 #pragma unroll
         for (int q = 0; q < BC_PER; ++q) {
-            const int i = tid + q * kDecThreads;
+            const int i = tid + q * THREADS;
             if (i < 2 * N) {
                 const int cc = HP + (i < N ? g * N + i : GN + g * N + (i - N));
                 T *cs = conv_state + ((size_t)b * Cc + cc) * (K - 1);
@@ -200,13 +200,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
     allow_dependents();
 }
 
-template <typename T, int N, int K, int ROWS>
+template <typename T, int N, int K, int ROWS, int THREADS>
 static cudaError_t decode_launch(float *ssm, void *conv_state, const void *xBC_t, const void *dt_t,
                                  const float *A_log, const float *D, const float *dt_bias, float dt_min,
                                  float dt_max, const void *conv_w, const void *conv_b, void *y_t,
                                  int B, int H, int P, int G, int *status, unsigned *counters, cudaStream_t st) {
     dim3 grid(H * P / ROWS, B);
-    return launch_pdl(decode_step_kernel<T, N, K, ROWS>, grid, dim3(kDecThreads), 0, st, ssm, (T *)conv_state,
+    return launch_pdl(decode_step_kernel<T, N, K, ROWS, THREADS>, grid, dim3(THREADS), 0, st, ssm, (T *)conv_state,
                       (const T *)xBC_t, (const T *)dt_t, A_log, D, dt_bias, dt_min, dt_max, (const T *)conv_w,
                       (const T *)conv_b, (T *)y_t, H, P, G, status, counters);
 }
@@ -217,9 +217,9 @@ static cudaError_t decode_rows(bool wide, float *ssm, void *conv_state, const vo
                                float dt_max, const void *conv_w, const void *conv_b, void *y_t, int B,
                                int H, int P, int G, int *status, unsigned *counters, cudaStream_t st) {
     if (wide)
-        return decode_launch<T, N, K, 64>(ssm, conv_state, xBC_t, dt_t, A_log, D, dt_bias, dt_min, dt_max,
+        return decode_launch<T, N, K, 64, 256>(ssm, conv_state, xBC_t, dt_t, A_log, D, dt_bias, dt_min, dt_max,
                                           conv_w, conv_b, y_t, B, H, P, G, status, counters, st);
-    return decode_launch<T, N, K, 16>(ssm, conv_state, xBC_t, dt_t, A_log, D, dt_bias, dt_min, dt_max,
+    return decode_launch<T, N, K, 16, 128>(ssm, conv_state, xBC_t, dt_t, A_log, D, dt_bias, dt_min, dt_max,
                                       conv_w, conv_b, y_t, B, H, P, G, status, counters, st);
 }
 

@@ -95,4 +95,8 @@ cudaError_t launch_causal_conv1d(int dtype, const void *xBC, const void *conv_w,
                                  const void *conv_b, void *out, void *conv_state_out, int B,
                                  int L, int Cc, int K, cudaStream_t st);
 
+// One warp waits on an mbarrier that nothing arrives at, for limit_us microseconds, and records
+// SSD_ERR_TIMEOUT in *status (the bounded-wait self-test).
+cudaError_t launch_selftest_wait(int *status, int limit_us, cudaStream_t st);
+
 }  // namespace ssd

@@ -61,13 +61,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Wait for the phase with the given parity to complete; false (and *status set) on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *status) {
+// Wait for the phase with the given parity to complete; false (and *status set) once
+// `limit_ns` of wall time have passed without it.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *status,
+                                          unsigned long long limit_ns = kWaitNs) {
     if (mbar_test(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     while (true) {
         if (mbar_test(bar, parity)) return true;
-        if (globaltimer() - t0 > kWaitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             if (status) atomicExch(status, SSD_ERR_TIMEOUT);
             return false;
         }

@@ -138,3 +138,9 @@ def test_decode_workspace_size():
 ])
 def test_conv_validation(args, want):
     assert L.ssd_causal_conv1d_fwd(*args) == want
+
+
+@pytest.mark.parametrize("status,limit_us", [(None, 1000), (A + 2, 1000), (A, 0), (A, 1000001)])
+def test_selftest_validation(status, limit_us):
+    # rejected before any launch, so it runs without a GPU
+    assert L.ssd_selftest_wait_timeout(status, limit_us, None) == INV
