@@ -63,14 +63,16 @@ __global__ void __launch_bounds__(256) state_pass_kernel(float *__restrict__ sta
 // same transposed layout in bf16 -- row-major [N][P], whose 128-byte-swizzled TMA tiles are the
 // MN-major B operand of O = C h_prev^T -- into a separate buffer.  h0 and h_final keep the
 // public [P][N] float32 layout.  Thread (n, p0..p0+3): one float4 load and one 8-byte store
-// per block, consecutive threads walking p then n, so every warp access is contiguous.
-__global__ void __launch_bounds__(256) state_pass_t_kernel(const float *__restrict__ statesT,
+// per block, consecutive threads walking p then n, so every warp access is contiguous.  Four
+// blocks' loads per round trip and at most 48 registers, so five CTAs share an SM and the
+// whole grid (B*H*P*N/4 threads: 640 CTAs for the 2.7B shape) is resident in one wave.
+__global__ void __launch_bounds__(256, 5) state_pass_t_kernel(const float *__restrict__ statesT,
                                                            const float *__restrict__ acs2,
                                                            const float *__restrict__ h0,
                                                            float *__restrict__ h_final,
                                                            __nv_bfloat16 *__restrict__ hT, int H,
                                                            int P, int N, int nc, int Q) {
-    constexpr int kAhead = 8;
+    constexpr int kAhead = 4;
     grid_dependency_wait();  // the block states come from the kernel before
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     const int p0 = (t * 4) % P, n = (t * 4) / P;
