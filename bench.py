@@ -675,8 +675,12 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": workload_config(),
+            # method-level count at the caller's chunk (256); the tensor-core path blocks the
+            # sequence in 128 tokens, which does fewer flops: both are reported
             "tflops": tflops, "tflops_frac": tflops * 1e12 / (peaks["bf16_tflops"] * 1e12) / world,
             "flops_per_layer_dense": flops_layer,
+            "tflops_executed_block128": prefill_flops(B, L, H, P, G, N, TC_BLOCK) * PF["layers"] * world
+                                        / (ms_step / 1e3) / 1e12,
             "flops_per_layer_causal": prefill_flops_causal(B, L, H, P, G, N, Q),
             "roofline": roof, "kernels": kernels, "decode": decode, "e2e": e2e,
             "cpu_baseline": cpu, "clocks": pf["clocks"],
