@@ -37,6 +37,14 @@
  *     launched and an SSD_ERR_* code is returned.  A failed launch returns
  *     SSD_ERR_CUDA; the CUDA error code is kept per host thread
  *     (ssd_last_cuda_error) and a sticky CUDA error is not cleared.  No kernel traps.
+ *   - The tensor-core prefill and the decode step are launched with programmatic
+ *     dependent launch: a kernel may be scheduled while the one before it in the stream
+ *     finishes, and reads and writes global memory only after that one has completed.
+ *     Setting SSD_PDL=0 in the environment (read once per process) launches them as
+ *     ordinary kernels.
+ *
+ * Version 2: ssd_decode_status and ssd_selftest_wait_timeout added; the decode workspace
+ * gained a status word (ssd_decode_workspace_size grew by 256 bytes).
  */
 #ifndef MAMBA_SSD_H
 #define MAMBA_SSD_H
@@ -102,6 +110,11 @@ SSD_API size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, 
  * Supported: H % G == 0, P == 64, N in {16, 32, 64, 128}, chunk in {64, 128, 256},
  * L >= 0, B >= 0.  Other valid shapes return SSD_ERR_UNSUPPORTED.  Calls sharing a
  * workspace must be ordered on one stream.
+ * Kernels: bf16 storage with N == 128 runs on the tcgen05 tensor cores, which compute the
+ * chunked form in 128-token blocks whatever `chunk` is (the decomposition is exact, only the
+ * rounding differs); float32 storage and the other N run on float32 CUDA-core kernels with
+ * the caller's chunk.  Setting SSD_PREFILL_KERNELS=simt in the environment (read once per
+ * process) sends every shape to the CUDA-core kernels.
  */
 SSD_API int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const void *Bm,
                        const void *Cm, const float *D, const float *dt_bias, float dt_min,

@@ -174,7 +174,7 @@ const char *ssd_status_string(int status) {
 
 int ssd_last_cuda_error(void) { return g_last_cuda_error; }
 
-int ssd_abi_version(void) { return 1; }
+int ssd_abi_version(void) { return 2; }
 
 size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, int N, int chunk,
                                      int dtype) {

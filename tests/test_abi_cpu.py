@@ -37,7 +37,7 @@ def test_status_strings_and_version():
     for s in range(6):
         assert L.ssd_status_string(s)
     assert L.ssd_status_string(99) == b"unknown status"
-    assert L.ssd_abi_version() >= 1
+    assert L.ssd_abi_version() == 2
     assert L.ssd_last_cuda_error() == 0
 
 
