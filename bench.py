@@ -511,7 +511,7 @@ def bench_decode(args, torch, ssd, device, rank, Bsz, steps):
             "kernel_gbs": decode_bytes(Bsz, H, P, G, N, K) / k_avg_s / 1e9 if kcnt else None}
 
 
-def bench_e2e(args, torch, ssd, device, steps):
+def bench_e2e(args, torch, ssd, device, rank, world, steps):
     """Prefill tokens/s through the public API with host buffers: every step copies each
     layer's inputs (x, dt, B, C) from pinned host memory to the device and reads y back.
 
@@ -519,7 +519,8 @@ def bench_e2e(args, torch, ssd, device, steps):
     stream-ordered API would: host-to-device copies on one stream, the prefill calls on a
     second, device-to-host copies on a third, over three device buffer sets, ordered by
     events.  The two copy directions and the kernels then run at the same time; the step
-    time is bounded by the slower PCIe direction."""
+    time is bounded by the slower PCIe direction.  Every rank runs its own replica; the value
+    is the tokens of all ranks over the slowest rank's time."""
     B, L, H, P, G, N, Q = PF["B"], PF["L"], PF["H"], PF["P"], PF["G"], PF["N"], PF["chunk"]
     n_layers = PF["layers"]
     nbuf = 3
@@ -567,14 +568,20 @@ def bench_e2e(args, torch, ssd, device, steps):
 
     step()
     torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(s_up)
     for _ in range(steps):
         step()
     end.record(s_down)  # the last read-back is the last operation of the timed steps
     torch.cuda.synchronize()
-    ms = start.elapsed_time(end) / steps
-    return {"value": B * L / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+    if world > 1:
+        torch.distributed.barrier()
+    ms = max_over_ranks(start.elapsed_time(end) / steps, world, device)
+    tokens = sum_over_ranks(B * L, world, device)
+    return {"value": tokens / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
             "h2d_gbs": h2d / (ms / 1e3) / 1e9, "d2h_gbs": d2h / (ms / 1e3) / 1e9,
             "note": ("per layer H2D of x, dt, B, C from pinned memory, prefill, D2H of y; "
@@ -659,8 +666,8 @@ def main():
             torch.cuda.empty_cache()
 
     e2e = None
-    if not args.no_e2e and rank == 0:
-        e2e = bench_e2e(args, torch, ssd, device, steps=max(1, min(args.steps, 3)))
+    if not args.no_e2e:  # every rank, the same collective steps in the same order
+        e2e = bench_e2e(args, torch, ssd, device, rank, world, steps=max(1, min(args.steps, 3)))
         torch.cuda.empty_cache()
 
     cpu = None
