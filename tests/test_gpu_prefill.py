@@ -75,6 +75,14 @@ def test_small_sweep(dtype, L, chunk, G, N, h0, bias):
     compare(inp, chunk, dtype, f"sweep {dtype} L{L} Q{chunk} G{G} N{N}")
 
 
+@pytest.mark.parametrize("B,L,H,G,h0", [(1, 32768, 8, 1, False), (2, 20000, 4, 2, True)])
+def test_long_sequence_tensor_cores(B, L, H, G, h0):
+    # hundreds of 128-token blocks: the state pass walks them all, the TMA coordinates and the
+    # per-CTA item ranges reach far into the workspace; the last block is ragged in the second
+    inp = S.prefill_inputs(B, L, H, 64, G, 128, dtype="bf16", seed=500 + L, h0=h0)
+    compare(inp, 256, "bf16", f"long sequence B{B} L{L} H{H} G{G}")
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_unclipped_dt_exercises_softplus(dtype):
     inp = S.prefill_inputs(1, 600, 8, 64, 2, 64, dtype=dtype, seed=77, h0=True,
