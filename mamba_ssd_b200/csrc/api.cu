@@ -49,7 +49,12 @@ cudaError_t timed_launch(KernelId id, cudaStream_t st, F &&launch) {
         a = pooled_event();
         b = pooled_event();
     }
-    if (!a || !b) return cudaErrorMemoryAllocation;
+    if (!a || !b) {  // give back whichever event was made
+        std::lock_guard<std::mutex> lk(g_timer_mu);
+        if (a) g_event_pool.push_back(a);
+        if (b) g_event_pool.push_back(b);
+        return cudaErrorMemoryAllocation;
+    }
     cudaEventRecord(a, st);
     const cudaError_t e = launch();
     cudaEventRecord(b, st);

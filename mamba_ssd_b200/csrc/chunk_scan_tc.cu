@@ -392,7 +392,8 @@ cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, 
                           (uint64_t)L * H * P * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
     const int grid = total < num_sms ? total : num_sms;
-    cudaFuncSetAttribute(chunk_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    e = raise_smem_limit<chunk_scan_tc_kernel>((int)kSmem);
+    if (e != cudaSuccess) return e;
     return launch_pdl(chunk_scan_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, tm_x, tm_b, tm_c, tm_h, tm_y,
                       dtf, acs, D, status, H, G, nk, total);
 }

@@ -257,8 +257,8 @@ static cudaError_t chunk_scan_n(const void *x, const void *Bm, const void *Cm, c
     const int nc = cdiv(L, chunk);
     dim3 grid(nc * (chunk / 64), H, B);
     constexpr size_t smem = chunk_scan_simt_smem<N>();
-    cudaFuncSetAttribute(chunk_scan_simt_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
+    const cudaError_t e = raise_smem_limit<chunk_scan_simt_kernel<T, N>>((int)smem);
+    if (e != cudaSuccess) return e;
     chunk_scan_simt_kernel<T, N><<<grid, 256, smem, st>>>((const T *)x, (const T *)Bm,
                                                           (const T *)Cm, dtf, acs, hprev, D,
                                                           (T *)y, L, H, G, chunk, nc);

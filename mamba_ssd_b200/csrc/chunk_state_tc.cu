@@ -376,7 +376,8 @@ cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const void *dt,
     e = make_tmap_f32_2d(&tm_s, states, (uint64_t)P, (uint64_t)total * N, (uint64_t)P * 4, 32, R);
     if (e != cudaSuccess) return e;
     const int grid = total < num_sms ? total : num_sms;
-    cudaFuncSetAttribute(chunk_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    e = raise_smem_limit<chunk_state_tc_kernel>((int)kSmem);
+    if (e != cudaSuccess) return e;
     return launch_pdl(chunk_state_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, tm_x, tm_b, tm_s,
                       (const __nv_bfloat16 *)dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, status, L, H, G, nk,
                       total);

@@ -78,7 +78,7 @@ template <typename T>
 static void decay_launch(dim3 grid, size_t smem, cudaStream_t st, const void *dt, const float *A_log,
                          const float *dt_bias, float dt_min, float dt_max, float *dtf, float *acs,
                          int *status, int L, int H, int chunk, int nc) {
-    cudaFuncSetAttribute(decay_prep_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // at most 8 x 257 floats (chunk <= 256): under the default 48 KB, no attribute needed
     decay_prep_kernel<T><<<grid, 256, smem, st>>>((const T *)dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, status,
                                                   L, H, chunk, nc);
 }

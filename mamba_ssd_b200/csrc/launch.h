@@ -5,7 +5,24 @@
 #include <cuda_runtime.h>
 #include <stddef.h>
 
+#include <atomic>
+
 namespace ssd {
+
+// A kernel's dynamic shared-memory limit, raised once per device (the attribute is per device;
+// raising it on every launch would cost a driver call each time).
+template <auto Kernel>
+cudaError_t raise_smem_limit(int bytes) {
+    static std::atomic<unsigned long long> done{0};  // bit d: raised on device d
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
 
 // Launches of the tensor-core prefill kernels use programmatic stream serialization (each may
 // be scheduled while the kernel before it finishes; the kernels order every global access
