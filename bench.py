@@ -588,6 +588,18 @@ def bench_e2e(args, torch, ssd, device, rank, world, steps):
                      "copies up, prefill and copies down on three streams over three buffer sets")}
 
 
+def decode_vs_recompute(prefill_ms, decode):
+    """The pages' headline comparison on this GPU: one cached decode step of the 64-layer
+    2.7B-shaped stack at batch 1 against recomputing the 4096-token prefix (the same stack's
+    prefill step, one batch row of 4096 tokens).  Both come from this run's measurements."""
+    b1 = decode.get("b1")
+    if not b1:
+        return None
+    step_ms = 1e3 / b1["steps_per_s"]
+    return {"context": PF["L"], "recompute_prefix_ms": prefill_ms, "cached_decode_step_ms": step_ms,
+            "speedup": prefill_ms / step_ms}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -690,6 +702,7 @@ def main():
                                         / (ms_step / 1e3) / 1e12,
             "flops_per_layer_causal": prefill_flops_causal(B, L, H, P, G, N, Q),
             "roofline": roof, "kernels": kernels, "decode": decode, "e2e": e2e,
+            "decode_vs_recompute": decode_vs_recompute(ms_step, decode),
             "cpu_baseline": cpu, "clocks": pf["clocks"],
             "gpu_launches": pf["launches_per_step"] * args.steps,
             "peaks": peaks,
