@@ -468,7 +468,7 @@ def bench_decode(args, torch, ssd, device, rank, Bsz, steps):
         layers.append(dict(ssm=ssm, conv=conv_state, w=conv_w, b=conv_b, A_log=A_log, D=D,
                            dt_bias=dt_bias, xs=xs, dts=dts, y=y))
     del pre_ws
-    ws = ssd.decode_workspace(Bsz, G, device)
+    ws = ssd.decode_workspace(Bsz, H, P, G, N, device)
     torch.cuda.synchronize()
 
     def run(step_range):
@@ -498,15 +498,20 @@ def bench_decode(args, torch, ssd, device, rank, Bsz, steps):
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
     with torch.cuda.stream(stream):
-        kt = kernel_times(torch, lib, lambda: run(range(min(steps, 8))), ["decode_step"])
+        kt = kernel_times(torch, lib, lambda: run(range(min(steps, 8))), ["decode_conv", "decode_step"])
     del graph
     bytes_step = DEC["layers"] * decode_bytes(Bsz, H, P, G, N, K)
     steps_s = steps / (ms / 1e3)
+    # one layer-step is two launches: the conv kernel, then the state update ("decode_step")
+    cms, ccnt = kt["decode_conv"]
     kms, kcnt = kt["decode_step"]
-    k_avg_s = kms / max(kcnt, 1) / 1e3
+    conv_s = cms / max(ccnt, 1) / 1e3
+    state_s = kms / max(kcnt, 1) / 1e3
+    k_avg_s = conv_s + state_s
     return {"batch": Bsz, "steps": steps, "layers": DEC["layers"], "ms": ms,
             "steps_per_s": steps_s, "gbs": bytes_step * steps_s / 1e9,
             "bytes_per_step": bytes_step, "launches": launches,
+            "conv_kernel_avg_us": conv_s * 1e6, "state_kernel_avg_us": state_s * 1e6,
             "kernel_avg_us": k_avg_s * 1e6,
             "kernel_gbs": decode_bytes(Bsz, H, P, G, N, K) / k_avg_s / 1e9 if kcnt else None}
 

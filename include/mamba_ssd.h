@@ -40,11 +40,16 @@
  *   - The tensor-core prefill and the decode step are launched with programmatic
  *     dependent launch: a kernel may be scheduled while the one before it in the stream
  *     finishes, and reads and writes global memory only after that one has completed.
- *     Setting SSD_PDL=0 in the environment (read once per process) launches them as
+ *     The one exception is the decode state kernel's reads of ssm_state, which begin while
+ *     the same call's conv kernel (which does not touch ssm_state) runs, but only after
+ *     every kernel enqueued before the call has completed.  Setting SSD_PDL=0 in the environment (read once per process) launches them as
  *     ordinary kernels.
  *
  * Version 2: ssd_decode_status and ssd_selftest_wait_timeout added; the decode workspace
  * gained a status word (ssd_decode_workspace_size grew by 256 bytes).
+ * Version 3: the decode step runs as two kernels; ssd_decode_workspace_size takes
+ * (B, H, P, G, N), the workspace holds the step's conv outputs instead of arrival counters
+ * and needs no zero-fill; the kernel timer knows "decode_conv".
  */
 #ifndef MAMBA_SSD_H
 #define MAMBA_SSD_H
@@ -165,23 +170,25 @@ SSD_API int ssd_chunk_scan_fwd_noalloc(const void *x, const void *dt, const floa
                                        void *stream);
 
 /*
- * Bytes of device workspace that ssd_decode_step needs (a multiple of 256).  The
- * workspace holds a status word and one arrival counter per (batch, group): it must be
- * zero-filled once before its first use, and every completed call leaves it zero-filled
- * again, so one zeroed workspace serves any number of consecutive calls on one stream.
+ * Bytes of device workspace that ssd_decode_step needs (a multiple of 256); 0 if an
+ * argument is not positive.  The workspace holds a status word, the step's conv outputs
+ * (B * (H*P + 2*G*N) floats) and its (dt, exp(dt*A)) pairs (B * H float2).  It needs no
+ * initialisation: every call writes what it reads.  One workspace serves any number of
+ * calls of the same or smaller shape that are ordered on one stream.
  */
-SSD_API size_t ssd_decode_workspace_size(int B, int G);
+SSD_API size_t ssd_decode_workspace_size(int B, int H, int P, int G, int N);
 
 /*
  * Diagnostic: synchronises `stream` and returns the status word the last ssd_decode_step
  * on `workspace` left; SSD_ERR_INVALID_ARG for a NULL workspace, SSD_ERR_CUDA if the stream
- * reported an error.  The decode kernel has no waits and always leaves SSD_OK; the word is
+ * reported an error.  The decode kernels have no waits and always leave SSD_OK; the word is
  * there so that a kernel with bounded waits can report SSD_ERR_TIMEOUT without an ABI change.
  */
 SSD_API int ssd_decode_status(const void *workspace, void *stream);
 
 /*
- * One cached decode step for one layer ([blog §2.1, §2.2]):
+ * One cached decode step for one layer ([blog §2.1, §2.2]), enqueued as two kernels on
+ * `stream` (the conv and conv-cache roll, then the state update):
  *   ssm_state  [B, H, P, N]   float  in/out: h <- exp(dt*A) h + dt x (outer) B
  *   conv_state [B, Cc, K-1]   dtype  in/out: the K-1 most recent raw xBC inputs,
  *                                    oldest first; rolled by one and the newest input
@@ -193,9 +200,13 @@ SSD_API int ssd_decode_status(const void *workspace, void *stream);
  *   conv_w     [Cc, K]        dtype  depthwise conv taps, tap K-1 multiplies the newest input
  *   conv_b     [Cc]           dtype  conv bias, NULL = 0
  *   y_t        [B, H, P]      dtype  output: y = h C + D x, with x, B, C = SiLU(conv + bias)
- *   workspace  ssd_decode_workspace_size(B, G) bytes, zero-filled before first use
- * Supported: H % G == 0, P % 16 == 0, N in {16, 32, 64, 128, 256}, 2 <= K <= 8.
- * Calls sharing a workspace must be ordered on one stream.
+ *   workspace  ssd_decode_workspace_size(B, H, P, G, N) bytes, 16-byte aligned
+ * Supported: H % G == 0, P % 16 == 0, N in {16, 32, 64, 128, 256}, 2 <= K <= 8,
+ * B <= 65535 (else SSD_ERR_UNSUPPORTED).  Calls sharing a workspace must be ordered on one
+ * stream.  With programmatic dependent launch (below), the state kernel starts reading
+ * ssm_state while the step's own conv kernel runs, after every kernel enqueued before the
+ * call has completed: ssm_state must not be written by anything running concurrently with
+ * the call, the same rule as for any other argument.
  */
 SSD_API int ssd_decode_step(float *ssm_state, void *conv_state, const void *xBC_t, const void *dt_t,
                     const float *A_log, const float *D, const float *dt_bias, float dt_min,
@@ -238,7 +249,8 @@ SSD_API int ssd_selftest_wait_timeout(int *status, int limit_us, void *stream);
  * ssd_kernel_timer_enable(1) makes every later kernel launch on this process record a
  * pair of CUDA events around itself on its own stream; ssd_kernel_timer_read(name, ...)
  * waits for the recorded events of kernel `name` ("decay_prep", "chunk_state",
- * "state_pass", "chunk_scan", "decode_step", "causal_conv1d"), returns the summed
+ * "state_pass", "chunk_scan", "decode_conv", "decode_step" (the decode state update),
+ * "causal_conv1d"), returns the summed
  * device time in milliseconds and the number of launches timed, and forgets them.
  * Do not enable the timer while a stream is being captured into a CUDA graph.
  * Returns SSD_OK, SSD_ERR_INVALID_ARG for an unknown name, SSD_ERR_CUDA on an event error.

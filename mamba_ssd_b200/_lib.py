@@ -33,7 +33,7 @@ SIGNATURES = {
     "ssd_chunk_scan_status": (_i, [_vp, _vp]),
     "ssd_chunk_scan_fwd_noalloc": (_i, [_vp, _vp, _fp, _vp, _vp, _fp, _fp, _f, _f, _fp, _vp, _fp]
                                    + [_i] * 8 + [_vp]),
-    "ssd_decode_workspace_size": (_sz, [_i, _i]),
+    "ssd_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "ssd_decode_status": (_i, [_vp, _vp]),
     "ssd_decode_step": (_i, [_fp, _vp, _vp, _vp, _fp, _fp, _fp, _f, _f, _vp, _vp, _vp]
                         + [_i] * 7 + [_vp, _sz, _vp]),

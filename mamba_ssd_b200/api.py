@@ -136,14 +136,15 @@ def ssd_selftest_wait_timeout(limit_us, device="cuda", stream=None):
     return int(status.item())
 
 
-def ssd_decode_workspace_size(B, G):
-    return int(_lib.lib().ssd_decode_workspace_size(B, G))
+def ssd_decode_workspace_size(B, H, P, G, N):
+    return int(_lib.lib().ssd_decode_workspace_size(B, H, P, G, N))
 
 
-def decode_workspace(B, G, device="cuda"):
-    """A zero-filled decode workspace (status word and arrival counters), reusable across
-    calls on one stream."""
-    return torch.zeros(max(ssd_decode_workspace_size(B, G), 256), device=device, dtype=torch.uint8)
+def decode_workspace(B, H, P, G, N, device="cuda"):
+    """A decode workspace (status word, the step's conv outputs and (dt, a) pairs), reusable
+    across calls of this shape or smaller on one stream.  Zero-filled only so that the status
+    word reads SSD_OK before the first call; the kernels need no initialisation."""
+    return torch.zeros(max(ssd_decode_workspace_size(B, H, P, G, N), 256), device=device, dtype=torch.uint8)
 
 
 def ssd_decode_step(ssm_state, conv_state, xBC_t, dt_t, A_log, D, dt_bias, conv_w, conv_b,
@@ -167,7 +168,7 @@ def ssd_decode_step(ssm_state, conv_state, xBC_t, dt_t, A_log, D, dt_bias, conv_
         y_t = torch.empty((Bsz, H, P), device=xBC_t.device, dtype=xBC_t.dtype)
     _need(y_t, "y_t", xBC_t.dtype, (Bsz, H, P))
     if workspace is None:
-        workspace = decode_workspace(Bsz, G, xBC_t.device)
+        workspace = decode_workspace(Bsz, H, P, G, N, xBC_t.device)
     s = _lib.lib().ssd_decode_step(
         _ptr(ssm_state), _ptr(conv_state), _ptr(xBC_t), _ptr(dt_t), _ptr(A_log), _ptr(D),
         _ptr(dt_bias), float(dt_min), float(dt_max), _ptr(conv_w), _ptr(conv_b), _ptr(y_t),

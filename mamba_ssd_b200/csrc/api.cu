@@ -17,9 +17,9 @@ namespace {
 thread_local int g_last_cuda_error = 0;
 
 // ---- profiling hooks: launch counter and optional per-kernel CUDA-event timing ----
-const char *const kKernelNames[] = {"decay_prep", "chunk_state", "state_pass",
-                                    "chunk_scan", "decode_step", "causal_conv1d"};
-enum KernelId { K_DECAY = 0, K_STATE, K_PASS, K_SCAN, K_DECODE, K_CONV, K_COUNT };
+const char *const kKernelNames[] = {"decay_prep", "chunk_state",   "state_pass", "chunk_scan",
+                                    "decode_step", "causal_conv1d", "decode_conv"};
+enum KernelId { K_DECAY = 0, K_STATE, K_PASS, K_SCAN, K_DECODE, K_CONV, K_DCONV, K_COUNT };
 
 std::atomic<long long> g_launches{0};
 std::atomic<int> g_timer_on{0};
@@ -179,7 +179,7 @@ const char *ssd_status_string(int status) {
 
 int ssd_last_cuda_error(void) { return g_last_cuda_error; }
 
-int ssd_abi_version(void) { return 2; }
+int ssd_abi_version(void) { return 3; }
 
 size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, int N, int chunk,
                                      int dtype) {
@@ -272,10 +272,17 @@ int ssd_chunk_scan_status(const void *workspace, void *stream) {
     return v;
 }
 
-// Decode workspace: a status word (256-byte slot), then one arrival counter per (batch, group).
-size_t ssd_decode_workspace_size(int B, int G) {
-    if (B <= 0 || G <= 0) return 0;
-    return 256 + ssd::align_up(sizeof(unsigned) * (size_t)B * G, 256);
+// Decode workspace: a status word (256-byte slot), then u [B][Cc] fp32 (the conv outputs of
+// the step), then (dt, a) [B][H] as float2; each part starts on a 256-byte boundary.
+namespace {
+size_t decode_u_bytes(int B, int H, int P, int G, int N) {
+    return ssd::align_up(sizeof(float) * (size_t)B * ((size_t)H * P + 2 * (size_t)G * N), 256);
+}
+}  // namespace
+
+size_t ssd_decode_workspace_size(int B, int H, int P, int G, int N) {
+    if (B <= 0 || H <= 0 || P <= 0 || G <= 0 || N <= 0) return 0;
+    return 256 + decode_u_bytes(B, H, P, G, N) + ssd::align_up(2 * sizeof(float) * (size_t)B * H, 256);
 }
 
 int ssd_decode_status(const void *workspace, void *stream) {
@@ -301,6 +308,7 @@ int ssd_decode_step(float *ssm_state, void *conv_state, const void *xBC_t, const
     if (P % 16 != 0) return SSD_ERR_UNSUPPORTED;
     if (!is_pow2_in(N, 16, 256)) return SSD_ERR_UNSUPPORTED;
     if (K < 2 || K > 8) return SSD_ERR_UNSUPPORTED;
+    if (B > 65535) return SSD_ERR_UNSUPPORTED;  // the batch is the grid's y dimension
     if (B == 0) return SSD_OK;
     if (!ssm_state || !conv_state || !xBC_t || !dt_t || !A_log || !conv_w || !y_t)
         return SSD_ERR_INVALID_ARG;
@@ -308,14 +316,20 @@ int ssd_decode_step(float *ssm_state, void *conv_state, const void *xBC_t, const
         !aligned16(A_log) || !aligned16(conv_w) || !aligned16(y_t) || !opt_aligned16(D) ||
         !opt_aligned16(dt_bias) || !opt_aligned16(conv_b))
         return SSD_ERR_INVALID_ARG;
-    if (!workspace || workspace_bytes < ssd_decode_workspace_size(B, G) || !aligned16(workspace))
+    if (!workspace || workspace_bytes < ssd_decode_workspace_size(B, H, P, G, N) || !aligned16(workspace))
         return SSD_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = timed_launch(K_DECODE, st, [&] {
-        return ssd::launch_decode_step(dtype, ssm_state, conv_state, xBC_t, dt_t, A_log, D, dt_bias,
-                                       dt_min, dt_max, conv_w, conv_b, y_t, B, H, P, G, N, K,
-                                       static_cast<int *>(workspace),
-                                       reinterpret_cast<unsigned *>(static_cast<char *>(workspace) + 256), st);
+    char *ws = static_cast<char *>(workspace);
+    float *u_ws = reinterpret_cast<float *>(ws + 256);
+    float2 *da_ws = reinterpret_cast<float2 *>(ws + 256 + decode_u_bytes(B, H, P, G, N));
+    cudaError_t e = timed_launch(K_DCONV, st, [&] {
+        return ssd::launch_decode_conv(dtype, conv_state, xBC_t, dt_t, A_log, dt_bias, dt_min, dt_max,
+                                       conv_w, conv_b, u_ws, da_ws, B, H, P, G, N, K, st);
+    });
+    if (e != cudaSuccess) return cuda_status(e);
+    e = timed_launch(K_DECODE, st, [&] {
+        return ssd::launch_decode_state(dtype, ssm_state, u_ws, da_ws, D, y_t, B, H, P, G, N,
+                                        static_cast<int *>(workspace), st);
     });
     return cuda_status(e);
 }

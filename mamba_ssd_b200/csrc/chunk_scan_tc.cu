@@ -130,6 +130,10 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
     const uint32_t tmem = *tmem_slot;
     // prologue done: from here on global memory is touched, after the previous kernel
     grid_dependency_wait();
+    dtf = after_wait(dtf);
+    acs = after_wait(acs);
+    D = after_wait(D);
+    status = after_wait(status);
 
     auto stage = [&](int j) { return smem + kOffStage + (uint32_t)(j % kStages) * kStageBytes; };
     // a bounded wait that gives up at once when another role has already timed out

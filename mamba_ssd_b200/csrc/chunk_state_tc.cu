@@ -119,6 +119,12 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     const uint32_t tmem = *tmem_slot;
     // prologue done: from here on global memory is touched, after the previous kernel
     grid_dependency_wait();
+    dt = after_wait(dt);
+    A_log = after_wait(A_log);
+    dt_bias = after_wait(dt_bias);
+    dtf = after_wait(dtf);
+    acs = after_wait(acs);
+    status = after_wait(status);
     // this call's status word starts clean (a later wait of the call may record a timeout)
     if (blockIdx.x == 0 && tid == 0) *status = SSD_OK;
 

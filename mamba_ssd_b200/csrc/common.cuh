@@ -63,6 +63,19 @@ __device__ __forceinline__ float warp_inclusive_sum(float v) {
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// after_wait(p): p, re-derived through an empty volatile asm placed after grid_dependency_wait().
+// A __restrict__ kernel parameter tells the compiler that nothing else writes its memory while
+// the kernel runs, which lets it move loads and stores through that pointer above the wait's
+// asm (the asm's memory clobber does not cover a pointer that never escaped) -- exactly wrong
+// when the previous kernel is still writing that memory.  An access through the returned
+// pointer depends on an asm that comes after the wait, so it cannot move above it.  Every
+// raw pointer a PDL kernel touches after its wait goes through this.
+template <typename T>
+__device__ __forceinline__ T *after_wait(T *p) {
+    asm volatile("" : "+l"(p));
+    return p;
+}
+
 __host__ __device__ constexpr inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ constexpr inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 

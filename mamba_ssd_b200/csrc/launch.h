@@ -101,12 +101,16 @@ cudaError_t launch_chunk_scan(int dtype, const void *x, const void *Bm, const vo
                               const float *D, void *y, int B, int L, int H, int G, int N,
                               int chunk, cudaStream_t st);
 
-cudaError_t launch_decode_step(int dtype, float *ssm_state, void *conv_state, const void *xBC_t,
-                               const void *dt_t, const float *A_log, const float *D,
-                               const float *dt_bias, float dt_min, float dt_max,
-                               const void *conv_w, const void *conv_b, void *y_t, int B, int H,
-                               int P, int G, int N, int K, int *status, unsigned *counters,
-                               cudaStream_t st);
+// One decode step is two launches: the conv kernel (conv, SiLU, conv-cache roll, dt and the
+// decay factor, into u_ws [B][Cc] fp32 and da_ws [B][H] (dt, a)), then the state kernel.
+cudaError_t launch_decode_conv(int dtype, void *conv_state, const void *xBC_t, const void *dt_t,
+                               const float *A_log, const float *dt_bias, float dt_min, float dt_max,
+                               const void *conv_w, const void *conv_b, float *u_ws, float2 *da_ws,
+                               int B, int H, int P, int G, int N, int K, cudaStream_t st);
+
+cudaError_t launch_decode_state(int dtype, float *ssm_state, const float *u_ws, const float2 *da_ws,
+                                const float *D, void *y_t, int B, int H, int P, int G, int N, int *status,
+                                cudaStream_t st);
 
 cudaError_t launch_causal_conv1d(int dtype, const void *xBC, const void *conv_w,
                                  const void *conv_b, void *out, void *conv_state_out, int B,

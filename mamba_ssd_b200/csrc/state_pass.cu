@@ -74,6 +74,11 @@ __global__ void __launch_bounds__(256, 5) state_pass_t_kernel(const float *__res
                                                            int P, int N, int nc, int Q) {
     constexpr int kAhead = 4;
     grid_dependency_wait();  // the block states come from the kernel before
+    statesT = after_wait(statesT);
+    acs2 = after_wait(acs2);
+    h0 = after_wait(h0);
+    h_final = after_wait(h_final);
+    hT = after_wait(hT);
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     const int p0 = (t * 4) % P, n = (t * 4) / P;
     const int h = blockIdx.y, b = blockIdx.z;

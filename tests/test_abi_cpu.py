@@ -37,7 +37,7 @@ def test_status_strings_and_version():
     for s in range(6):
         assert L.ssd_status_string(s)
     assert L.ssd_status_string(99) == b"unknown status"
-    assert L.ssd_abi_version() == 2
+    assert L.ssd_abi_version() == 3
     assert L.ssd_last_cuda_error() == 0
 
 
@@ -113,6 +113,7 @@ def decode(**kw):
     (dict(H=81, G=2), INV), (dict(G=0), INV), (dict(dtype=2), INV), (dict(dt_min=0.2), INV),
     (dict(P=24), UNS), (dict(N=48), UNS), (dict(N=512), UNS), (dict(K=1), UNS), (dict(K=9), UNS),
     (dict(ws=None), WS), (dict(ws_bytes=0), WS), (dict(B=300), WS),
+    (dict(ws_bytes=22527), WS), (dict(B=70000), UNS),
     (dict(B=0), OK),
 ])
 def test_decode_validation(kw, want):
@@ -120,12 +121,14 @@ def test_decode_validation(kw, want):
 
 
 def test_decode_workspace_size():
-    # a 256-byte status slot, then one 4-byte counter per (batch, group) rounded up to 256
-    assert L.ssd_decode_workspace_size(1, 1) == 512
-    assert L.ssd_decode_workspace_size(16, 8) == 768
-    assert L.ssd_decode_workspace_size(64, 2) == 768
-    assert L.ssd_decode_workspace_size(65, 2) == 1024
-    assert L.ssd_decode_workspace_size(0, 1) == 0
+    # a 256-byte status slot, then B*(H*P + 2*G*N) floats and B*H float2, each part rounded
+    # up to 256 bytes:  (B, H, P, G, N) -> 256 + u + (dt, a)
+    assert L.ssd_decode_workspace_size(1, 80, 64, 1, 128) == 256 + 21504 + 768
+    assert L.ssd_decode_workspace_size(16, 80, 64, 1, 128) == 256 + 344064 + 10240
+    assert L.ssd_decode_workspace_size(3, 2, 16, 1, 16) == 256 + 768 + 256
+    assert L.ssd_decode_workspace_size(0, 80, 64, 1, 128) == 0
+    assert L.ssd_decode_workspace_size(1, 0, 64, 1, 128) == 0
+    assert L.ssd_decode_workspace_size(1, 80, 64, 1, -1) == 0
 
 
 @pytest.mark.parametrize("args,want", [

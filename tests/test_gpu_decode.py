@@ -44,9 +44,10 @@ def test_decode_steps_match_oracle(dtype, B, H, G, N, K):
     tok0 = S.decode_token_inputs(B, H, P, G, N, K, dtype=dtype, seed=4)
     state = {"ssm": dev(tok0["ssm_state"][0]).clone(), "conv": dev(tok0["conv_state"][0]).clone()}
     ref_ssm, ref_conv = tok0["ssm_state"][1], tok0["conv_state"][1]
-    ws = ssd.decode_workspace(B, G)
+    ws = ssd.decode_workspace(B, H, P, G, N)
+    ws.fill_(0xA5)  # the workspace needs no initialisation: every call writes what it reads
     pf = f64(prm)
-    for step in range(3):  # consecutive steps reuse one workspace (counters reset)
+    for step in range(3):  # consecutive steps reuse one workspace
         tok = S.decode_token_inputs(B, H, P, G, N, K, dtype=dtype, seed=10 + step)
         y = gpu_decode(state, prm, tok, H, P, G, N, ws)
         torch.cuda.synchronize()
@@ -58,8 +59,7 @@ def test_decode_steps_match_oracle(dtype, B, H, G, N, K):
         check_close(host64(state["ssm"]), ref_ssm, dtype, "h", f"step {step} state")
         # the conv cache only moves raw inputs: exact
         np.testing.assert_array_equal(host64(state["conv"]), ref_conv)
-    assert ssd.ssd_decode_status(ws) == 0, "a bounded wait inside the decode kernel gave up"
-    assert torch.count_nonzero(ws) == 0, "status word and arrival counters must be left at zero"
+    assert ssd.ssd_decode_status(ws) == 0, "the decode kernels must leave the status word at SSD_OK"
 
 
 @pytest.mark.parametrize("dtype,B,L,Cc,K", [
@@ -133,7 +133,7 @@ def test_prefill_then_decode_pipeline(B, steps):
                                         pf["dt_bias"], pf["dt_min"], pf["dt_max"], None)
     torch.cuda.synchronize()
     check_close(host64(ssm), h64, "bf16", "h", "state after prefill")
-    ws = ssd.decode_workspace(B, G)
+    ws = ssd.decode_workspace(B, H, P, G, N)
     ys = []
     for j in range(steps):
         t = L + j
