@@ -329,8 +329,9 @@ def workload_config():
 # ---------------------------------------------------------------------------------------
 # GPU legs
 # ---------------------------------------------------------------------------------------
-def make_prefill_layers(torch, device, layers, rank):
-    H, P, G, N, B, L = PF["H"], PF["P"], PF["G"], PF["N"], PF["B"], PF["L"]
+def make_prefill_layers(torch, device, layers, rank, L=None):
+    H, P, G, N, B = PF["H"], PF["P"], PF["G"], PF["N"], PF["B"]
+    L = PF["L"] if L is None else L
     out = []
     for layer in range(layers):
         g = torch.Generator(device=device)
@@ -516,6 +517,80 @@ def bench_decode(args, torch, ssd, device, rank, Bsz, steps):
             "kernel_gbs": decode_bytes(Bsz, H, P, G, N, K) / k_avg_s / 1e9 if kcnt else None}
 
 
+def bench_context_sweep(torch, ssd, device, rank, contexts=(1024, 4096, 16384), dec_steps=16):
+    """Cached decode against recomputing the prefix, by context length L.  For each L: the
+    64-layer stack's prefill over L tokens (what a model without the cache recomputes for
+    every generated token), then B = 1 decode steps of the same stack starting from the
+    states that prefill left.  A decode step reads and writes the fixed-size state only, so
+    its time must not grow with L while the recompute grows linearly."""
+    H, P, G, N, K = PF["H"], PF["P"], PF["G"], PF["N"], DEC["K"]
+    Cc = H * P + 2 * G * N
+    bf = torch.bfloat16
+    stream = torch.cuda.Stream(device=device)
+    rows = []
+    for L in contexts:
+        layers = make_prefill_layers(torch, device, PF["layers"], rank, L=L)
+        ws = torch.empty(ssd.ssd_chunk_scan_workspace_size(1, L, H, P, G, N, PF["chunk"], bf),
+                         device=device, dtype=torch.uint8)
+        with torch.cuda.stream(stream):
+            for lay in layers:
+                prefill_call(ssd, lay, ws)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for lay in layers:
+                prefill_call(ssd, lay, ws)
+        pre_ms = time_graph(torch, graph, stream, reps=3)
+        del graph
+        # decode from the states the prefill left; per-layer conv taps, cache and tokens
+        g = torch.Generator(device=device)
+        g.manual_seed(DEC["seed"] * 7 + L)
+        scale = torch.ones(Cc, device=device)
+        scale[H * P:] = 1.0 / math.sqrt(N)
+        dec = []
+        for lay in layers:
+            dec.append(dict(
+                ssm=lay["hf"], A_log=lay["A_log"], D=lay["D"], dt_bias=lay["dt_bias"],
+                conv=(torch.randn((1, Cc, K - 1), generator=g, device=device) * scale[:, None]).to(bf),
+                w=((torch.rand((Cc, K), generator=g, device=device) * 2 - 1) / math.sqrt(K)).to(bf),
+                b=((torch.rand((Cc,), generator=g, device=device) * 2 - 1) / math.sqrt(K)).to(bf),
+                xs=(torch.randn((dec_steps, 1, Cc), generator=g, device=device) * scale).to(bf),
+                dts=(torch.randn((dec_steps, 1, H), generator=g, device=device) - 2.0).to(bf),
+                y=torch.empty((dec_steps, 1, H, P), device=device, dtype=bf)))
+            for k in ("x", "dt", "Bm", "Cm", "y"):
+                del lay[k]
+        del ws
+        dws = ssd.decode_workspace(1, H, P, G, N, device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for s in range(dec_steps):
+                for d in dec:
+                    ssd.ssd_decode_step(d["ssm"], d["conv"], d["xs"][s], d["dts"][s], d["A_log"], d["D"],
+                                        d["dt_bias"], d["w"], d["b"], H, P, G, N, dt_min=1e-3, dt_max=0.1,
+                                        y_t=d["y"][s], workspace=dws)
+        dec_ms = time_graph(torch, graph, stream, reps=3) / dec_steps
+        del graph, dec, layers
+        torch.cuda.synchronize()
+        rows.append({"L": L, "recompute_ms": pre_ms, "decode_step_ms": dec_ms, "speedup": pre_ms / dec_ms})
+    return rows
+
+
+def time_graph(torch, graph, stream, reps):
+    """Median CUDA-event time of `reps` replays of a captured graph, after one warm-up."""
+    graph.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    return sorted(times)[len(times) // 2]
+
+
 def bench_e2e(args, torch, ssd, device, rank, world, steps):
     """Prefill tokens/s through the public API with host buffers: every step copies each
     layer's inputs (x, dt, B, C) from pinned host memory to the device and reads y back.
@@ -593,7 +668,7 @@ def bench_e2e(args, torch, ssd, device, rank, world, steps):
                      "copies up, prefill and copies down on three streams over three buffer sets")}
 
 
-def decode_vs_recompute(prefill_ms, decode):
+def decode_vs_recompute(prefill_ms, decode, by_context=None):
     """The pages' headline comparison on this GPU: one cached decode step of the 64-layer
     2.7B-shaped stack at batch 1 against recomputing the 4096-token prefix (the same stack's
     prefill step, one batch row of 4096 tokens).  Both come from this run's measurements."""
@@ -602,7 +677,7 @@ def decode_vs_recompute(prefill_ms, decode):
         return None
     step_ms = 1e3 / b1["steps_per_s"]
     return {"context": PF["L"], "recompute_prefix_ms": prefill_ms, "cached_decode_step_ms": step_ms,
-            "speedup": prefill_ms / step_ms}
+            "speedup": prefill_ms / step_ms, "by_context": by_context}
 
 
 def main():
@@ -672,7 +747,7 @@ def main():
             kernels[n].update(algorithmic_bytes=kb, gbs=kb / avg / 1e9, frac=kb / avg / 1e9 / peaks["hbm_gbs"],
                               traffic=measured_traffic(n))
 
-    decode = {}
+    decode, by_context = {}, None
     if not args.no_decode:
         for bsz in (1, 16):
             r = bench_decode(args, torch, ssd, device, rank, bsz, DEC["steps"])
@@ -681,6 +756,8 @@ def main():
                 r["kernel_gbs_frac"] = r["kernel_gbs"] / peaks["hbm_gbs"]
             decode[f"b{bsz}"] = r
             torch.cuda.empty_cache()
+        by_context = bench_context_sweep(torch, ssd, device, rank)
+        torch.cuda.empty_cache()
 
     e2e = None
     if not args.no_e2e:  # every rank, the same collective steps in the same order
@@ -707,7 +784,7 @@ def main():
                                         / (ms_step / 1e3) / 1e12,
             "flops_per_layer_causal": prefill_flops_causal(B, L, H, P, G, N, Q),
             "roofline": roof, "kernels": kernels, "decode": decode, "e2e": e2e,
-            "decode_vs_recompute": decode_vs_recompute(ms_step, decode),
+            "decode_vs_recompute": decode_vs_recompute(ms_step, decode, by_context),
             "cpu_baseline": cpu, "clocks": pf["clocks"],
             "gpu_launches": pf["launches_per_step"] * args.steps,
             "peaks": peaks,

@@ -112,7 +112,7 @@ SSD_API size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, 
  *   workspace, workspace_bytes         >= ssd_chunk_scan_workspace_size(...), 256-byte
  *                                      aligned, contents on entry irrelevant; it is
  *                                      scratch for this call only
- * Supported: H % G == 0, P == 64, N in {16, 32, 64, 128}, chunk in {64, 128, 256},
+ * Supported: H % G == 0, P == 64, N in {16, 32, 64, 128}, chunk in {64, 128, 256, 512},
  * L >= 0, B >= 0.  Other valid shapes return SSD_ERR_UNSUPPORTED.  Calls sharing a
  * workspace must be ordered on one stream.
  * Kernels: bf16 storage with N == 128 runs on the tcgen05 tensor cores, which compute the

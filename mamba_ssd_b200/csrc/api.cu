@@ -116,7 +116,7 @@ int check_prefill_shape(int B, int L, int H, int P, int G, int N, int chunk, int
     if (H % G != 0) return SSD_ERR_INVALID_ARG;
     if (P != 64) return SSD_ERR_UNSUPPORTED;
     if (N != 16 && N != 32 && N != 64 && N != 128) return SSD_ERR_UNSUPPORTED;
-    if (chunk != 64 && chunk != 128 && chunk != 256) return SSD_ERR_UNSUPPORTED;
+    if (chunk != 64 && chunk != 128 && chunk != 256 && chunk != 512) return SSD_ERR_UNSUPPORTED;
     return SSD_OK;
 }
 

@@ -33,8 +33,8 @@ __global__ void __launch_bounds__(256) decay_prep_kernel(
     if (status && c == 0 && b == 0 && blockIdx.z == 0 && threadIdx.x == 0) *status = SSD_OK;
     const int nh = min(8, H - hb);
     const int ld = Q + 1;
-    // Q * 8 slots over 256 threads: at most 8 per thread (Q <= 256), loads issued together
-    constexpr int kPer = 8;
+    // Q * 8 slots over 256 threads: at most 16 per thread (Q <= 512), loads issued together
+    constexpr int kPer = 16;
     float raw[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
@@ -78,7 +78,7 @@ template <typename T>
 static void decay_launch(dim3 grid, size_t smem, cudaStream_t st, const void *dt, const float *A_log,
                          const float *dt_bias, float dt_min, float dt_max, float *dtf, float *acs,
                          int *status, int L, int H, int chunk, int nc) {
-    // at most 8 x 257 floats (chunk <= 256): under the default 48 KB, no attribute needed
+    // at most 8 x 513 floats (chunk <= 512): under the default 48 KB, no attribute needed
     decay_prep_kernel<T><<<grid, 256, smem, st>>>((const T *)dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, status,
                                                   L, H, chunk, nc);
 }

@@ -89,7 +89,7 @@ def prefill(**kw):
     (dict(B=-1), INV), (dict(L=-3), INV), (dict(H=0), INV), (dict(G=3), INV), (dict(dtype=7), INV),
     (dict(dt_min=0.5, dt_max=0.1), INV), (dict(dt_min=-1.0), INV), (dict(dt_max=float("nan")), INV),
     (dict(P=32), UNS), (dict(N=48), UNS), (dict(N=256), UNS), (dict(chunk=100), UNS),
-    (dict(chunk=512), UNS),
+    (dict(chunk=1024), UNS), (dict(chunk=32), UNS),
     (dict(ws=None), WS), (dict(ws_bytes=1024), WS), (dict(ws=A + 16), WS),
     (dict(B=0), OK),
 ])

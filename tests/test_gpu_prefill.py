@@ -75,6 +75,18 @@ def test_small_sweep(dtype, L, chunk, G, N, h0, bias):
     compare(inp, chunk, dtype, f"sweep {dtype} L{L} Q{chunk} G{G} N{N}")
 
 
+@pytest.mark.parametrize("dtype,L,G,N,h0", [
+    ("f32", 1, 1, 16, False), ("f32", 511, 2, 64, True), ("bf16", 513, 1, 32, False),
+    ("bf16", 1500, 2, 16, True), ("f32", 9000, 1, 64, True), ("bf16", 9000, 1, 128, False),
+])
+def test_chunk_512(dtype, L, G, N, h0):
+    # chunk 512, the size suggested beyond 8k tokens: one and several chunks, ragged tails.
+    # bf16 N = 128 runs on the tensor cores (128-token blocks whatever the chunk); the others
+    # run the CUDA-core kernels with 512-token chunks.
+    inp = S.prefill_inputs(1, L, 4, 64, G, N, dtype=dtype, seed=500 + L + N, h0=h0)
+    compare(inp, 512, dtype, f"chunk 512 {dtype} L{L} G{G} N{N}")
+
+
 @pytest.mark.parametrize("B,L,H,G,h0", [(1, 32768, 8, 1, False), (2, 20000, 4, 2, True)])
 def test_long_sequence_tensor_cores(B, L, H, G, h0):
     # hundreds of 128-token blocks: the state pass walks them all, the TMA coordinates and the
