@@ -10,13 +10,17 @@ Forms:
   forms.ssd_dense             quadratic dual form M x (numpy, tiny inputs)
   native.causal_conv1d        prefix depthwise conv + SiLU and the cache it leaves (C)
   native.decode_step          one cached decode step (C)
+  block.gated_rmsnorm         the block step after the scan: y * SiLU(z), RMS-normalised per
+                              token and norm group, scaled per channel (numpy)
 
 Parity status: every function here is pinned by closed forms, invariants or
-brute force in tests/test_oracle_pins.py; none is "parity unpinned".
+brute force in tests/test_oracle_pins.py and tests/test_oracle_norm.py; none is
+"parity unpinned".
 """
 from .native import (ssd_scan_sequential, causal_conv1d, decode_step, dt_value,
                      max_threads, set_threads)
 from .forms import ssd_chunked, ssd_dense, discretise, softplus
+from .block import gated_rmsnorm, silu
 
 __all__ = ["ssd_scan_sequential", "causal_conv1d", "decode_step", "dt_value", "max_threads",
-           "set_threads", "ssd_chunked", "ssd_dense", "discretise", "softplus"]
+           "set_threads", "ssd_chunked", "ssd_dense", "discretise", "softplus", "gated_rmsnorm", "silu"]
