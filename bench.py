@@ -575,6 +575,41 @@ def bench_context_sweep(torch, ssd, device, rank, contexts=(1024, 4096, 16384), 
     return rows
 
 
+def bench_block_norm(torch, ssd, device, peaks, launches=64, buffers=8):
+    """The block step after the scan on the 2.7B shape: gated RMS norm of one layer's scan
+    output (4096 tokens x 5120 channels, bf16, one norm group).  `launches` calls cycle over
+    `buffers` distinct (y, z, out) sets (1 GB in all, far above L2), captured in one graph;
+    reported per launch against the measured copy bandwidth."""
+    T, C = PF["B"] * PF["L"], PF["H"] * PF["P"]
+    bf = torch.bfloat16
+    g = torch.Generator(device=device)
+    g.manual_seed(PF["seed"] + 77)
+    sets = [dict(y=torch.randn((T, C), generator=g, device=device).to(bf),
+                 z=torch.randn((T, C), generator=g, device=device).to(bf),
+                 out=torch.empty((T, C), device=device, dtype=bf)) for _ in range(buffers)]
+    w = torch.rand((C,), generator=g, device=device) + 0.5
+    stream = torch.cuda.Stream(device=device)
+
+    def run():
+        for i in range(launches):
+            st = sets[i % buffers]
+            ssd.ssd_gated_rmsnorm_fwd(st["y"], st["z"], w, n_groups=1, eps=1e-5, out=st["out"])
+
+    with torch.cuda.stream(stream):
+        run()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        run()
+    ms = time_graph(torch, graph, stream, reps=5)
+    del graph, sets
+    per_launch_s = ms / launches / 1e3
+    nbytes = 3 * T * C * 2 + C * 4
+    return {"kernel": "gated_rmsnorm", "workload": f"{T} tokens x {C} channels, bf16, 1 norm group",
+            "avg_us": per_launch_s * 1e6, "algorithmic_bytes": nbytes, "gbs": nbytes / per_launch_s / 1e9,
+            "frac": nbytes / per_launch_s / 1e9 / peaks["hbm_gbs"], "launches_timed": launches}
+
+
 def time_graph(torch, graph, stream, reps):
     """Median CUDA-event time of `reps` replays of a captured graph, after one warm-up."""
     graph.replay()
@@ -758,6 +793,8 @@ def main():
             torch.cuda.empty_cache()
         by_context = bench_context_sweep(torch, ssd, device, rank)
         torch.cuda.empty_cache()
+    block_steps = {"gated_rmsnorm": bench_block_norm(torch, ssd, device, peaks)}
+    torch.cuda.empty_cache()
 
     e2e = None
     if not args.no_e2e:  # every rank, the same collective steps in the same order
@@ -785,6 +822,7 @@ def main():
             "flops_per_layer_causal": prefill_flops_causal(B, L, H, P, G, N, Q),
             "roofline": roof, "kernels": kernels, "decode": decode, "e2e": e2e,
             "decode_vs_recompute": decode_vs_recompute(ms_step, decode, by_context),
+            "block_steps": block_steps,
             "cpu_baseline": cpu, "clocks": pf["clocks"],
             "gpu_launches": pf["launches_per_step"] * args.steps,
             "peaks": peaks,

@@ -49,7 +49,7 @@
  * gained a status word (ssd_decode_workspace_size grew by 256 bytes).
  * Version 3: the decode step runs as two kernels; ssd_decode_workspace_size takes
  * (B, H, P, G, N), the workspace holds the step's conv outputs instead of arrival counters
- * and needs no zero-fill; the kernel timer knows "decode_conv".
+ * and needs no zero-fill; the kernel timer knows "decode_conv"; ssd_gated_rmsnorm_fwd added.
  */
 #ifndef MAMBA_SSD_H
 #define MAMBA_SSD_H
@@ -230,6 +230,26 @@ SSD_API int ssd_causal_conv1d_fwd(const void *xBC, const void *conv_w, const voi
                           void *stream);
 
 /*
+ * Gated RMS norm, the block step after the scan ([blog §4.1]: a norm takes its variance in
+ * float32 even for bf16 inputs; the gate and the per-group RMS are the Mamba-2 block's norm,
+ * which the pages name without spelling out):
+ *   g   = y * SiLU(z)
+ *   out = g / sqrt(mean over the channels of its group of g^2 + eps) * w
+ *   y, z  [T, C]  dtype  the scan output and the gate input, T tokens of C channels (for a
+ *                        prefill output y[B, L, H, P]: T = B*L, C = H*P)
+ *   w     [C]     float  per-channel scale
+ *   out   [T, C]  dtype  must not overlap y or z
+ *   n_groups             norm groups per token: C / n_groups consecutive channels each
+ * The mean square is accumulated in float32.  Supported: C % n_groups == 0,
+ * C / n_groups a multiple of 8 and at most 32768, n_groups <= 65535, eps >= 0 and finite.
+ * Pointers 16-byte aligned.  Errors: SSD_ERR_INVALID_ARG (bad sizes, eps, dtype, pointers),
+ * SSD_ERR_UNSUPPORTED (group size), SSD_ERR_CUDA.  T == 0 is a no-op.  Launched with
+ * programmatic dependent launch like the prefill kernels.
+ */
+SSD_API int ssd_gated_rmsnorm_fwd(const void *y, const void *z, const float *w, void *out, int T, int C,
+                                  int n_groups, float eps, int dtype, void *stream);
+
+/*
  * Self-test of the bounded waits (no counterpart in the pages; the failure path of the
  * tensor-core kernels).  Launches one warp that waits, with the same bounded-wait code the
  * prefill kernels use, on an mbarrier that no thread ever arrives at, giving up after
@@ -250,7 +270,7 @@ SSD_API int ssd_selftest_wait_timeout(int *status, int limit_us, void *stream);
  * pair of CUDA events around itself on its own stream; ssd_kernel_timer_read(name, ...)
  * waits for the recorded events of kernel `name` ("decay_prep", "chunk_state",
  * "state_pass", "chunk_scan", "decode_conv", "decode_step" (the decode state update),
- * "causal_conv1d"), returns the summed
+ * "causal_conv1d", "gated_rmsnorm"), returns the summed
  * device time in milliseconds and the number of launches timed, and forgets them.
  * Do not enable the timer while a stream is being captured into a CUDA graph.
  * Returns SSD_OK, SSD_ERR_INVALID_ARG for an unknown name, SSD_ERR_CUDA on an event error.

@@ -39,6 +39,7 @@ SIGNATURES = {
                         + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_causal_conv1d_fwd": (_i, [_vp] * 5 + [_i] * 5 + [_vp]),
     "ssd_selftest_wait_timeout": (_i, [_vp, _i, _vp]),
+    "ssd_gated_rmsnorm_fwd": (_i, [_vp, _vp, _fp, _vp, _i, _i, _i, _f, _i, _vp]),
     "ssd_kernel_launch_count": (ctypes.c_longlong, []),
     "ssd_kernel_timer_enable": (_i, [_i]),
     "ssd_kernel_timer_read": (_i, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),

@@ -195,3 +195,22 @@ def ssd_causal_conv1d_fwd(xBC, conv_w, conv_b=None, out=None, conv_state_out=Non
         code, _stream(stream))
     check(s, "ssd_causal_conv1d_fwd")
     return out, conv_state_out
+
+
+def ssd_gated_rmsnorm_fwd(y, z, w, n_groups=1, eps=1e-5, out=None, stream=None):
+    """Gated RMS norm over the last axis: y * SiLU(z), RMS-normalised per token and norm
+    group (fp32 mean square), times w.  y and z share shape [..., C] and dtype; w is [C]
+    float32.  Returns out (same shape and dtype as y)."""
+    C = y.shape[-1]
+    code = _dtype_code(y)
+    _need(y, "y")
+    _need(z, "z", y.dtype, tuple(y.shape))
+    _need(w, "w", torch.float32, (C,))
+    if out is None:
+        out = torch.empty_like(y)
+    _need(out, "out", y.dtype, tuple(y.shape))
+    T = y.numel() // C if C else 0
+    s = _lib.lib().ssd_gated_rmsnorm_fwd(_ptr(y), _ptr(z), _ptr(w), _ptr(out), T, C, int(n_groups),
+                                         float(eps), code, _stream(stream))
+    check(s, "ssd_gated_rmsnorm_fwd")
+    return out

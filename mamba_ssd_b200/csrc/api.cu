@@ -17,9 +17,9 @@ namespace {
 thread_local int g_last_cuda_error = 0;
 
 // ---- profiling hooks: launch counter and optional per-kernel CUDA-event timing ----
-const char *const kKernelNames[] = {"decay_prep", "chunk_state",   "state_pass", "chunk_scan",
-                                    "decode_step", "causal_conv1d", "decode_conv"};
-enum KernelId { K_DECAY = 0, K_STATE, K_PASS, K_SCAN, K_DECODE, K_CONV, K_DCONV, K_COUNT };
+const char *const kKernelNames[] = {"decay_prep",  "chunk_state",   "state_pass",  "chunk_scan",
+                                    "decode_step", "causal_conv1d", "decode_conv", "gated_rmsnorm"};
+enum KernelId { K_DECAY = 0, K_STATE, K_PASS, K_SCAN, K_DECODE, K_CONV, K_DCONV, K_NORM, K_COUNT };
 
 std::atomic<long long> g_launches{0};
 std::atomic<int> g_timer_on{0};
@@ -354,6 +354,22 @@ int ssd_causal_conv1d_fwd(const void *xBC, const void *conv_w, const void *conv_
     return cuda_status(timed_launch(K_CONV, st, [&] {
         return ssd::launch_causal_conv1d(dtype, xBC, conv_w, conv_b, out, conv_state_out, B, L, Cc, K,
                                          st);
+    }));
+}
+
+int ssd_gated_rmsnorm_fwd(const void *y, const void *z, const float *w, void *out, int T, int C,
+                          int n_groups, float eps, int dtype, void *stream) {
+    if (T < 0 || C <= 0 || n_groups <= 0 || C % n_groups != 0) return SSD_ERR_INVALID_ARG;
+    if (dtype != SSD_DTYPE_F32 && dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !(eps < INFINITY)) return SSD_ERR_INVALID_ARG;  // also rejects NaN
+    const int GS = C / n_groups;
+    if (GS % 8 != 0 || GS > 32768 || n_groups > 65535) return SSD_ERR_UNSUPPORTED;
+    if (T == 0) return SSD_OK;
+    if (!y || !z || !w || !out || !aligned16(y) || !aligned16(z) || !aligned16(w) || !aligned16(out))
+        return SSD_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return cuda_status(timed_launch(K_NORM, st, [&] {
+        return ssd::launch_gated_rmsnorm(dtype, y, z, w, out, T, C, n_groups, eps, st);
     }));
 }
 

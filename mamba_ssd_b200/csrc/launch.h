@@ -112,6 +112,11 @@ cudaError_t launch_decode_state(int dtype, float *ssm_state, const float *u_ws, 
                                 const float *D, void *y_t, int B, int H, int P, int G, int N, int *status,
                                 cudaStream_t st);
 
+// Gated RMS norm over T_rows tokens of C channels in n_groups groups (C / n_groups channels
+// each, a multiple of the 16-byte vector and at most 32768).
+cudaError_t launch_gated_rmsnorm(int dtype, const void *y, const void *z, const float *w, void *out, int T_rows,
+                                 int C, int n_groups, float eps, cudaStream_t st);
+
 cudaError_t launch_causal_conv1d(int dtype, const void *xBC, const void *conv_w,
                                  const void *conv_b, void *out, void *conv_state_out, int B,
                                  int L, int Cc, int K, cudaStream_t st);

@@ -12,6 +12,8 @@ Distributions (the workload descriptions; N(mu, var) is mean and *variance*):
   h0 = 0, or N(0, 0.1) for the batched workload that exercises state carry-in.
 Decode (2.7B-shaped): raw xBC with the x channels N(0, 1) and the B/C channels
 N(0, 1/N); depthwise conv weight and bias ~ U(-1/sqrt(K), 1/sqrt(K)).
+Gated norm after the scan: y ~ N(0, 1) (the scale of the scan output), gate input
+z ~ N(0, 1), per-channel weight w ~ U(0.5, 1.5) in fp32.
 """
 from __future__ import annotations
 
@@ -23,7 +25,7 @@ import numpy as np
 __all__ = [
     "PrefillShape", "DecodeShape", "PREFILL_WORKLOADS", "DECODE_WORKLOAD",
     "bf16_bits", "bf16_bits_to_f64", "to_storage", "prefill_inputs",
-    "decode_params", "decode_token_inputs", "raw_xbc_sequence", "layer_seed",
+    "decode_params", "decode_token_inputs", "raw_xbc_sequence", "layer_seed", "norm_inputs",
 ]
 
 
@@ -202,3 +204,15 @@ def decode_token_inputs(B, H, P, G, N, K, dtype="bf16", seed=0, state_std=0.1):
         "ssm_state": _f32(ssm), "conv_state": to_storage(conv_state, dtype),
         "xBC_t": to_storage(xbc, dtype), "dt_t": to_storage(dt, dtype),
     }
+
+
+# ----------------------------------------------------------------------------------
+# gated norm inputs
+# ----------------------------------------------------------------------------------
+def norm_inputs(T, C, dtype="bf16", seed=0):
+    """y[T, C] and z[T, C] in the storage dtype, w[C] fp32."""
+    rng = np.random.default_rng(seed)
+    y = rng.standard_normal((T, C), dtype=np.float32)
+    z = rng.standard_normal((T, C), dtype=np.float32)
+    w = rng.uniform(0.5, 1.5, size=C).astype(np.float32)
+    return {"y": to_storage(y, dtype), "z": to_storage(z, dtype), "w": _f32(w)}

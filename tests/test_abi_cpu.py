@@ -147,3 +147,23 @@ def test_conv_validation(args, want):
 def test_selftest_validation(status, limit_us):
     # rejected before any launch, so it runs without a GPU
     assert L.ssd_selftest_wait_timeout(status, limit_us, None) == INV
+
+
+def norm(**kw):
+    a = dict(y=A, z=A, w=A, out=A, T=4096, C=5120, G=1, eps=1e-5, dtype=BF16, stream=None)
+    a.update(kw)
+    return L.ssd_gated_rmsnorm_fwd(a["y"], a["z"], a["w"], a["out"], a["T"], a["C"], a["G"], a["eps"],
+                                   a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(y=None), INV), (dict(z=MIS), INV), (dict(w=None), INV), (dict(out=MIS), INV),
+    (dict(T=-1), INV), (dict(C=0), INV), (dict(G=0), INV), (dict(C=5120, G=3), INV),
+    (dict(dtype=5), INV), (dict(eps=-1e-3), INV), (dict(eps=float("nan")), INV),
+    (dict(eps=float("inf")), INV),
+    (dict(C=12), UNS), (dict(C=65536, G=1), UNS), (dict(C=640 * 70000, G=70000), UNS),
+    (dict(T=0), OK), (dict(T=0, y=None, z=None, out=None), OK),
+])
+def test_norm_validation(kw, want):
+    # every case is decided before a launch, so it runs without a GPU
+    assert norm(**kw) == want
