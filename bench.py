@@ -610,6 +610,44 @@ def bench_block_norm(torch, ssd, device, peaks, launches=64, buffers=8):
             "frac": nbytes / per_launch_s / 1e9 / peaks["hbm_gbs"], "launches_timed": launches}
 
 
+def bench_block_conv(torch, ssd, device, peaks, launches=64, buffers=8):
+    """The block step before the scan on the 2.7B shape: causal depthwise conv1d + SiLU of
+    one layer's raw xBC (4096 tokens x 5376 channels, K = 4, bf16) and the conv cache it
+    leaves.  `launches` calls cycle over `buffers` distinct input/output sets (700 MB in all,
+    far above L2), captured in one graph; reported per launch against the measured copy
+    bandwidth."""
+    B, L, H, P, G, N, K = PF["B"], PF["L"], PF["H"], PF["P"], PF["G"], PF["N"], DEC["K"]
+    Cc = H * P + 2 * G * N
+    bf = torch.bfloat16
+    g = torch.Generator(device=device)
+    g.manual_seed(PF["seed"] + 78)
+    sets = [dict(x=torch.randn((B, L, Cc), generator=g, device=device).to(bf),
+                 out=torch.empty((B, L, Cc), device=device, dtype=bf),
+                 cs=torch.empty((B, Cc, K - 1), device=device, dtype=bf)) for _ in range(buffers)]
+    w = ((torch.rand((Cc, K), generator=g, device=device) * 2 - 1) / math.sqrt(K)).to(bf)
+    bias = ((torch.rand((Cc,), generator=g, device=device) * 2 - 1) / math.sqrt(K)).to(bf)
+    stream = torch.cuda.Stream(device=device)
+
+    def run():
+        for i in range(launches):
+            st = sets[i % buffers]
+            ssd.ssd_causal_conv1d_fwd(st["x"], w, bias, out=st["out"], conv_state_out=st["cs"])
+
+    with torch.cuda.stream(stream):
+        run()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        run()
+    ms = time_graph(torch, graph, stream, reps=5)
+    del graph, sets
+    per_launch_s = ms / launches / 1e3
+    nbytes = 2 * B * L * Cc * 2 + B * Cc * (K - 1) * 2 + Cc * (K + 1) * 2
+    return {"kernel": "causal_conv1d", "workload": f"B={B}, L={L}, {Cc} channels, K={K}, bf16",
+            "avg_us": per_launch_s * 1e6, "algorithmic_bytes": nbytes, "gbs": nbytes / per_launch_s / 1e9,
+            "frac": nbytes / per_launch_s / 1e9 / peaks["hbm_gbs"], "launches_timed": launches}
+
+
 def time_graph(torch, graph, stream, reps):
     """Median CUDA-event time of `reps` replays of a captured graph, after one warm-up."""
     graph.replay()
@@ -793,7 +831,8 @@ def main():
             torch.cuda.empty_cache()
         by_context = bench_context_sweep(torch, ssd, device, rank)
         torch.cuda.empty_cache()
-    block_steps = {"gated_rmsnorm": bench_block_norm(torch, ssd, device, peaks)}
+    block_steps = {"causal_conv1d": bench_block_conv(torch, ssd, device, peaks),
+                   "gated_rmsnorm": bench_block_norm(torch, ssd, device, peaks)}
     torch.cuda.empty_cache()
 
     e2e = None

@@ -223,7 +223,8 @@ SSD_API int ssd_decode_step(float *ssm_state, void *conv_state, const void *xBC_
  *   out            [B, L, Cc]  dtype  SiLU(sum_k w[c,k] xBC[t-K+1+k, c] + b[c])
  *   conv_state_out [B, Cc, K-1] dtype the last K-1 raw inputs, oldest first, zeros
  *                                     before the start; NULL = not written
- * Supported: 2 <= K <= 8, Cc % 8 == 0, L >= 0.
+ * Supported: 2 <= K <= 8, Cc % 8 == 0, 0 <= L <= 2097120, B <= 65535.  Launched with
+ * programmatic dependent launch.
  */
 SSD_API int ssd_causal_conv1d_fwd(const void *xBC, const void *conv_w, const void *conv_b, void *out,
                           void *conv_state_out, int B, int L, int Cc, int K, int dtype,

@@ -340,6 +340,7 @@ int ssd_causal_conv1d_fwd(const void *xBC, const void *conv_w, const void *conv_
     if (B < 0 || L < 0 || Cc <= 0 || K <= 0) return SSD_ERR_INVALID_ARG;
     if (dtype != SSD_DTYPE_F32 && dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
     if (K < 2 || K > 8 || Cc % 8 != 0) return SSD_ERR_UNSUPPORTED;
+    if (B > 65535 || L > 65535 * 32) return SSD_ERR_UNSUPPORTED;  // grid z; 32-token strips on grid y
     if (B == 0) return SSD_OK;
     if (!conv_w || !aligned16(conv_w) || !opt_aligned16(conv_b) || !opt_aligned16(conv_state_out))
         return SSD_ERR_INVALID_ARG;

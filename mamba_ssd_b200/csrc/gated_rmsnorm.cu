@@ -34,13 +34,6 @@ struct Vec16<float> {
     static constexpr int n = 4;
 };
 
-// SiLU with the fast hardware exponential and division (relative error about 1e-6, far inside
-// the output's own rounding).  The exponent is clamped at 80 so that 1 + e^-z stays below
-// 2^126, where __fdividef is exact to a few ulp; below z = -80 the gate is 0 to within 1e-33.
-__device__ __forceinline__ float silu_fast(float z) {
-    return __fdividef(z, 1.f + __expf(fminf(-z, 80.f)));
-}
-
 template <typename T>
 __global__ void __launch_bounds__(kNormThreads) gated_rmsnorm_kernel(const T *__restrict__ y,
                                                                      const T *__restrict__ z,

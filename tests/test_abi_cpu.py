@@ -138,6 +138,8 @@ def test_decode_workspace_size():
     ((None, A, A, A, A, 1, 16, 64, 4, BF16, None), INV),
     ((A, A, A, A, A, 0, 16, 64, 4, BF16, None), OK),
     ((None, A, A, None, None, 2, 0, 64, 4, F32, None), OK),
+    ((A, A, A, A, A, 1, 65535 * 32 + 1, 64, 4, BF16, None), UNS),
+    ((A, A, A, A, A, 65536, 16, 64, 4, BF16, None), UNS),
 ])
 def test_conv_validation(args, want):
     assert L.ssd_causal_conv1d_fwd(*args) == want

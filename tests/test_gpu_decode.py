@@ -65,6 +65,9 @@ def test_decode_steps_match_oracle(dtype, B, H, G, N, K):
 @pytest.mark.parametrize("dtype,B,L,Cc,K", [
     ("bf16", 1, 1, 64, 4), ("bf16", 2, 2, 72, 4), ("f32", 1, 3, 16, 4), ("f32", 2, 70, 40, 3),
     ("bf16", 1, 4096, 5376, 4), ("bf16", 3, 130, 128, 2),
+    # 32-token strips and 8-token request batches: lengths around both, every K up to 8
+    ("bf16", 2, 33, 64, 8), ("f32", 1, 65, 24, 5), ("bf16", 1, 31, 8, 6), ("bf16", 1, 32, 16, 7),
+    ("f32", 2, 9, 32, 2),
 ])
 def test_causal_conv_matches_oracle(dtype, B, L, Cc, K):
     rng = np.random.default_rng(L + Cc)
@@ -75,6 +78,18 @@ def test_causal_conv_matches_oracle(dtype, B, L, Cc, K):
     torch.cuda.synchronize()
     out_ref, cs_ref = oracle.causal_conv1d(xbc[1], w[1], b[1])
     check_close(host64(out), out_ref, dtype, "y", "conv out")
+    np.testing.assert_array_equal(host64(cs), cs_ref)
+
+
+def test_causal_conv_without_bias():
+    rng = np.random.default_rng(5)
+    B, L, Cc, K = 2, 40, 48, 4
+    xbc = S.to_storage(rng.standard_normal((B, L, Cc), dtype=np.float32), "bf16")
+    w = S.to_storage(rng.uniform(-0.5, 0.5, (Cc, K)).astype(np.float32), "bf16")
+    out, cs = ssd.ssd_causal_conv1d_fwd(dev(xbc[0]), dev(w[0]), None)
+    torch.cuda.synchronize()
+    out_ref, cs_ref = oracle.causal_conv1d(xbc[1], w[1], None)
+    check_close(host64(out), out_ref, "bf16", "y", "conv out, no bias")
     np.testing.assert_array_equal(host64(cs), cs_ref)
 
 
