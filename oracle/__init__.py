@@ -12,6 +12,8 @@ Forms:
   native.decode_step          one cached decode step (C)
   block.gated_rmsnorm         the block step after the scan: y * SiLU(z), RMS-normalised per
                               token and norm group, scaled per channel (numpy)
+  varlen.ssd_scan_varlen      sequences of different lengths packed into one token stream,
+                              each scanned on its own (a loop over native.ssd_scan_sequential)
 
 Parity status: every function here is pinned by closed forms, invariants or
 brute force in tests/test_oracle_pins.py and tests/test_oracle_norm.py; none is
@@ -21,6 +23,8 @@ from .native import (ssd_scan_sequential, causal_conv1d, decode_step, dt_value,
                      max_threads, set_threads)
 from .forms import ssd_chunked, ssd_dense, discretise, softplus
 from .block import gated_rmsnorm, silu
+from .varlen import ssd_scan_varlen
 
 __all__ = ["ssd_scan_sequential", "causal_conv1d", "decode_step", "dt_value", "max_threads",
-           "set_threads", "ssd_chunked", "ssd_dense", "discretise", "softplus", "gated_rmsnorm", "silu"]
+           "set_threads", "ssd_chunked", "ssd_dense", "discretise", "softplus", "gated_rmsnorm", "silu",
+           "ssd_scan_varlen"]
