@@ -49,7 +49,8 @@
  * gained a status word (ssd_decode_workspace_size grew by 256 bytes).
  * Version 3: the decode step runs as two kernels; ssd_decode_workspace_size takes
  * (B, H, P, G, N), the workspace holds the step's conv outputs instead of arrival counters
- * and needs no zero-fill; the kernel timer knows "decode_conv"; ssd_gated_rmsnorm_fwd added.
+ * and needs no zero-fill; the kernel timer knows "decode_conv"; ssd_gated_rmsnorm_fwd and
+ * ssd_chunk_scan_varlen_fwd added.
  */
 #ifndef MAMBA_SSD_H
 #define MAMBA_SSD_H
@@ -126,6 +127,30 @@ SSD_API int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log
                        float dt_max, const float *h0, void *y, float *h_final, int B, int L,
                        int H, int P, int G, int N, int chunk, int dtype, void *workspace,
                        size_t workspace_bytes, void *stream);
+
+/*
+ * Varlen prefill: n_seq sequences of different lengths packed into one token stream, each
+ * scanned on its own, as in the chunked prefill above ([blog §1.1]: the state is passed
+ * along one sequence only).  Sequence i owns tokens cu_seqlens[i] .. cu_seqlens[i+1]-1:
+ *   x [T, H, P], dt [T, H], Bm, Cm [T, G, N], y [T, H, P]   packed, T = cu_seqlens[n_seq]
+ *   cu_seqlens  HOST array of n_seq + 1 ints, cu_seqlens[0] = 0, never decreasing (empty
+ *               sequences allowed: their h_final is their h0, or 0)
+ *   h0, h_final [n_seq, H, P, N] float, each nullable
+ *   A_log, D, dt_bias, dt_min, dt_max, chunk, dtype   as for ssd_chunk_scan_fwd
+ *   workspace   ssd_chunk_scan_workspace_size(1, longest length, H, P, G, N, chunk, dtype)
+ *               bytes, 256-byte aligned, shared by the sequences
+ * Each sequence runs the prefill kernels of ssd_chunk_scan_fwd with B = 1, in order on
+ * `stream` (three launches per non-empty sequence on the tensor-core path).  Everything is
+ * validated before the first launch: SSD_ERR_INVALID_ARG for bad cu_seqlens or pointers,
+ * SSD_ERR_UNSUPPORTED for a shape ssd_chunk_scan_fwd would not take or a sequence whose dt
+ * rows would not start 16-byte aligned (never when H * sizeof(element) is a multiple of 16),
+ * SSD_ERR_WORKSPACE.  A CUDA launch error stops the loop and is returned as SSD_ERR_CUDA.
+ */
+SSD_API int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float *A_log, const void *Bm,
+                                      const void *Cm, const float *D, const float *dt_bias, float dt_min,
+                                      float dt_max, const float *h0, void *y, float *h_final,
+                                      const int *cu_seqlens, int n_seq, int H, int P, int G, int N, int chunk,
+                                      int dtype, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Diagnostic: waits for `stream` to finish (this call synchronises, unlike every other

@@ -85,6 +85,47 @@ def ssd_chunk_scan_fwd(x, dt, A_log, Bm, Cm, D=None, chunk=256, h0=None, dt_bias
     return y, h_final
 
 
+def ssd_chunk_scan_varlen_fwd(x, dt, A_log, Bm, Cm, cu_seqlens, D=None, chunk=256, h0=None,
+                              dt_bias=None, dt_min=0.0, dt_max=math.inf, y=None, h_final=None,
+                              workspace=None, want_h_final=True, stream=None):
+    """Varlen SSD prefill: x [T,H,P], dt [T,H], Bm/Cm [T,G,N] hold n sequences packed by the
+    cumulative lengths cu_seqlens (n+1 ints on the host: a list, numpy array or CPU tensor).
+    Returns (y [T,H,P], h_final [n,H,P,N] or None)."""
+    import ctypes
+    cu = [int(v) for v in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    n = len(cu) - 1
+    T, H, P = x.shape
+    G, N = Bm.shape[1], Bm.shape[2]
+    code = _dtype_code(x)
+    _need(x, "x")
+    _need(dt, "dt", x.dtype, (T, H))
+    _need(Bm, "Bm", x.dtype, (T, G, N))
+    _need(Cm, "Cm", x.dtype, (T, G, N))
+    _need(A_log, "A_log", torch.float32, (H,))
+    _need(D, "D", torch.float32, (H,))
+    _need(dt_bias, "dt_bias", torch.float32, (H,))
+    _need(h0, "h0", torch.float32, (n, H, P, N))
+    if n < 0 or cu[-1] != T:
+        raise ValueError(f"cu_seqlens must end at the token count {T}")
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", x.dtype, x.shape)
+    if h_final is None and want_h_final:
+        h_final = torch.empty((n, H, P, N), device=x.device, dtype=torch.float32)
+    _need(h_final, "h_final", torch.float32, (n, H, P, N))
+    longest = max([b - a for a, b in zip(cu, cu[1:])] + [0])
+    need = _lib.lib().ssd_chunk_scan_workspace_size(1, longest, H, P, G, N, chunk, code)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), device=x.device, dtype=torch.uint8)
+    cu_arr = (ctypes.c_int * len(cu))(*cu)
+    s = _lib.lib().ssd_chunk_scan_varlen_fwd(
+        _ptr(x), _ptr(dt), _ptr(A_log), _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(dt_bias),
+        float(dt_min), float(dt_max), _ptr(h0), _ptr(y), _ptr(h_final), ctypes.cast(cu_arr, ctypes.c_void_p),
+        n, H, P, G, N, int(chunk), code, _ptr(workspace), workspace.numel(), _stream(stream))
+    check(s, "ssd_chunk_scan_varlen_fwd")
+    return y, h_final
+
+
 def ssd_chunk_scan_fwd_noalloc(x, dt, A_log, Bm, Cm, D=None, chunk=256, h0=None, dt_bias=None,
                                dt_min=0.0, dt_max=math.inf, y=None, h_final=None, stream=None):
     """ssd_chunk_scan_fwd whose scratch is the library's built-in device array (no workspace

@@ -262,6 +262,59 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
     return SSD_OK;
 }
 
+int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float *A_log, const void *Bm,
+                              const void *Cm, const float *D, const float *dt_bias, float dt_min,
+                              float dt_max, const float *h0, void *y, float *h_final,
+                              const int *cu_seqlens, int n_seq, int H, int P, int G, int N, int chunk,
+                              int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    if (n_seq < 0 || (n_seq > 0 && !cu_seqlens)) return SSD_ERR_INVALID_ARG;
+    if (n_seq == 0) return SSD_OK;
+    // lengths: start at 0, never decrease
+    if (cu_seqlens[0] != 0) return SSD_ERR_INVALID_ARG;
+    int max_len = 0;
+    for (int i = 0; i < n_seq; ++i) {
+        const int len = cu_seqlens[i + 1] - cu_seqlens[i];
+        if (cu_seqlens[i + 1] < cu_seqlens[i]) return SSD_ERR_INVALID_ARG;
+        if (len > max_len) max_len = len;
+    }
+    int s = check_prefill_shape(1, max_len, H, P, G, N, chunk, dtype);
+    if (s != SSD_OK) return s;
+    if ((s = check_dt_range(dt_min, dt_max)) != SSD_OK) return s;
+    const size_t e = dtype == SSD_DTYPE_BF16 ? 2 : 4;
+    const bool any_tokens = cu_seqlens[n_seq] > 0;
+    if (!A_log || !aligned16(A_log) || !opt_aligned16(D) || !opt_aligned16(dt_bias) || !opt_aligned16(h0) ||
+        !opt_aligned16(h_final))
+        return SSD_ERR_INVALID_ARG;
+    if (any_tokens && (!x || !dt || !Bm || !Cm || !y || !aligned16(x) || !aligned16(dt) || !aligned16(Bm) ||
+                       !aligned16(Cm) || !aligned16(y)))
+        return SSD_ERR_INVALID_ARG;
+    // every sequence's rows must start on a 16-byte boundary (x, y, B, C always do for the
+    // supported P and N; dt does when H * e is a multiple of 16 or the offsets happen to be)
+    for (int i = 0; i < n_seq; ++i)
+        if (((size_t)cu_seqlens[i] * H * e) % 16 != 0 || ((size_t)cu_seqlens[i] * G * N * e) % 16 != 0)
+            return SSD_ERR_UNSUPPORTED;
+    const size_t need = ssd::prefill_query_bytes(1, max_len, H, P, N, chunk, dtype);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return SSD_ERR_WORKSPACE;
+    // every argument is valid: run each sequence through the prefill, in order on the stream,
+    // sharing the workspace (each call's kernels start after the previous call's have ended)
+    const size_t state = (size_t)H * P * N;
+    for (int i = 0; i < n_seq; ++i) {
+        const size_t t0 = (size_t)cu_seqlens[i];
+        const int len = cu_seqlens[i + 1] - cu_seqlens[i];
+        const char *xb = static_cast<const char *>(x), *dtb = static_cast<const char *>(dt);
+        const char *bb = static_cast<const char *>(Bm), *cb = static_cast<const char *>(Cm);
+        char *yb = static_cast<char *>(y);
+        s = ssd_chunk_scan_fwd(xb ? xb + t0 * H * P * e : nullptr, dtb ? dtb + t0 * H * e : nullptr, A_log,
+                               bb ? bb + t0 * G * N * e : nullptr, cb ? cb + t0 * G * N * e : nullptr, D, dt_bias,
+                               dt_min, dt_max, h0 ? h0 + i * state : nullptr, yb ? yb + t0 * H * P * e : nullptr,
+                               h_final ? h_final + i * state : nullptr, 1, len, H, P, G, N, chunk, dtype, workspace,
+                               workspace_bytes, stream);
+        if (s != SSD_OK) return s;
+    }
+    return SSD_OK;
+}
+
 int ssd_chunk_scan_status(const void *workspace, void *stream) {
     if (!workspace) return SSD_ERR_INVALID_ARG;
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

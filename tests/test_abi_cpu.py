@@ -169,3 +169,29 @@ def norm(**kw):
 def test_norm_validation(kw, want):
     # every case is decided before a launch, so it runs without a GPU
     assert norm(**kw) == want
+
+
+def varlen(cu, **kw):
+    a = dict(x=A, dt=A, A_log=A, Bm=A, Cm=A, D=None, dt_bias=None, dt_min=1e-3, dt_max=0.1, h0=None, y=A,
+             hf=None, n=len(cu) - 1 if cu is not None else 1, H=80, P=64, G=1, N=128, chunk=256, dtype=BF16,
+             ws=A * 256, ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    arr = (ctypes.c_int * len(cu))(*cu) if cu is not None else None
+    return L.ssd_chunk_scan_varlen_fwd(a["x"], a["dt"], a["A_log"], a["Bm"], a["Cm"], a["D"], a["dt_bias"],
+                                       a["dt_min"], a["dt_max"], a["h0"], a["y"], a["hf"],
+                                       ctypes.cast(arr, ctypes.c_void_p) if arr is not None else None, a["n"],
+                                       a["H"], a["P"], a["G"], a["N"], a["chunk"], a["dtype"], a["ws"],
+                                       a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("cu,kw,want", [
+    (None, {}, INV), ([0, 5], dict(n=-1), INV), ([1, 5], {}, INV), ([0, 5, 3], {}, INV),
+    ([0, 5], dict(x=None), INV), ([0, 5], dict(dt=MIS), INV), ([0, 5], dict(A_log=None), INV),
+    ([0, 5], dict(P=32), UNS), ([0, 5], dict(chunk=100), UNS),
+    ([0, 1, 4], dict(H=4), UNS),          # bf16 dt rows of sequence 1 would start 8 bytes in
+    ([0, 5], dict(ws=None), WS), ([0, 5], dict(ws_bytes=256), WS), ([0, 5], dict(ws=A + 16), WS),
+    ([0], {}, OK), ([0, 0, 0], dict(x=None, dt=None, Bm=None, Cm=None, y=None, n=0), OK),
+])
+def test_varlen_validation(cu, kw, want):
+    # every case is decided before a launch, so it runs without a GPU
+    assert varlen(cu, **kw) == want
