@@ -9,7 +9,10 @@ layers (batch 1, 4096 tokens, H=80, P=64, G=1, N=128, chunk 256, bf16 storage, f
 state).  `value` is prefill tokens/s of the whole stack: B*L / (time of one step).  The
 same run also measures the cached decode step of the 2.7B-shaped decode workload (64
 layers, ssm_state [B,80,64,128] fp32 + conv_state [B,5376,3] bf16, B in {1, 16}, 64
-steps from a state built by a 4096-token prefill) and reports it under "decode".
+steps from a state built by a 4096-token prefill) and reports it under "decode";
+"decode_vs_recompute" divides the prefill of a 1024-, 4096- and 16384-token prefix through
+the stack by one batch-1 decode step of it; "block_steps" times the prefix conv and the
+gated RMS norm on one 2.7B layer.
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and
 torch.cuda.synchronize(), timed with CUDA events on the launching stream; the step is
