@@ -195,3 +195,28 @@ def varlen(cu, **kw):
 def test_varlen_validation(cu, kw, want):
     # every case is decided before a launch, so it runs without a GPU
     assert varlen(cu, **kw) == want
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    # the boundary is a C ABI: the header compiles as C99 and as C++17, and a C program links
+    # against the library and calls it (host-only entry points: no GPU needed)
+    import shutil
+    import subprocess
+    if not shutil.which("gcc"):
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text('#include "mamba_ssd.h"\n#include <stdio.h>\n'
+                   "int main(void) {\n"
+                   "  size_t ws = ssd_decode_workspace_size(16, 80, 64, 1, 128);\n"
+                   "  printf(\"%d %zu %s\\n\", ssd_abi_version(), ws, ssd_status_string(SSD_OK));\n"
+                   "  return ws == 256 + 344064 + 10240 ? 0 : 1;\n}\n")
+    inc = os.path.join(ROOT, "include")
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    for cmd in (["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only", f"-I{inc}", str(src)],
+                ["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-x", "c++", f"-I{inc}", str(src)]):
+        subprocess.run(cmd, check=True)
+    exe = tmp_path / "use"
+    subprocess.run(["gcc", "-std=c99", f"-I{inc}", str(src), f"-L{libdir}", "-lmamba_ssd",
+                    f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out[0] == str(L.ssd_abi_version())
