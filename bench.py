@@ -78,8 +78,10 @@ def prefill_bytes(B, L, H, P, G, N, e=2, h0=False):
     return B * L * (2 * H * P * e + 2 * G * N * e + H * e) + (2 if h0 else 1) * B * H * P * N * 4
 
 
-# Per-kernel algorithmic bytes of the tensor-core prefill (128-token blocks): every tensor a
-# kernel must read or write once, the workspace tensors passed between the kernels included.
+# Per-kernel bytes the tensor-core prefill (128-token blocks) must move: every tensor a kernel
+# reads or writes once, the workspace tensors passed between the kernels included.  These are
+# design costs, not algorithmic work: the algorithmic (method-level) work of the prefill is
+# prefill_flops / prefill_bytes above, and each kernel's share of it is KERNEL_METHOD_FLOPS.
 TC_BLOCK = 128
 
 
@@ -106,6 +108,11 @@ def chunk_scan_bytes(B, L, H, P, G, N, e=2):
 
 
 KERNEL_BYTES = {"chunk_state": chunk_state_bytes, "state_pass": state_pass_bytes, "chunk_scan": chunk_scan_bytes}
+# Each kernel's share of the method-level flops (the dense-tile count of prefill_flops at the
+# caller's chunk): the block state is step a3 (2HNP per token), the chunk scan steps a2 + a5 (CB once
+# per group, the masked product, C h_prev); the state pass is step a4, a scan with no
+# contraction.
+KERNEL_METHOD_FLOPS = {"chunk_state": chunk_state_flops, "chunk_scan": chunk_scan_flops}
 # The sources a kernel's DRAM-traffic capture depends on: a capture is used only while these
 # files are byte-identical to the ones it was taken with.
 KERNEL_SOURCES = {"chunk_state": ["chunk_state_tc.cu"], "state_pass": ["state_pass.cu"],
@@ -266,19 +273,66 @@ def oracle_step(f):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(min_seconds=10.0, max_reps=50):
-    import oracle
-    f = oracle_layer_inputs()
+def _timed_reps(fn, min_seconds, max_reps, min_reps=1):
     times = []
     t_start = time.perf_counter()
-    while len(times) < max_reps and (time.perf_counter() - t_start) < min_seconds:
-        times.append(oracle_step(f))
-    per_layer = statistics.median(times)
+    while len(times) < max_reps and (len(times) < min_reps or (time.perf_counter() - t_start) < min_seconds):
+        times.append(fn())
+    return statistics.median(times), len(times)
+
+
+def oracle_decode_inputs(Bsz):
+    """One 2.7B-shaped decode layer's cache and token (seeded), as the oracle consumes them."""
+    import ssd_synth as S
+    H, P, G, N, K = DEC["H"], DEC["P"], DEC["G"], DEC["N"], DEC["K"]
+    prm = S.decode_params(H, P, G, N, K, seed=S.layer_seed(DEC["seed"], 0))
+    tok = S.decode_token_inputs(Bsz, H, P, G, N, K, dtype="bf16", seed=S.layer_seed(DEC["seed"], 900))
+    f = {k: (v[1] if isinstance(v, tuple) else v) for k, v in {**prm, **tok}.items()}
+    return f
+
+
+def oracle_decode_layer(f):
+    import oracle
+    H, P, G, N = DEC["H"], DEC["P"], DEC["G"], DEC["N"]
+    t0 = time.perf_counter()
+    oracle.decode_step(f["ssm_state"], f["conv_state"], f["xBC_t"], f["dt_t"], f["A_log"], f["D"], f["dt_bias"],
+                       f["dt_min"], f["dt_max"], f["conv_w"], f["conv_b"], H, P, G, N)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(min_seconds=10.0, max_reps=50):
+    """The fp64 oracle on this host's cores: the prefill recurrence (the headline leg) on all
+    cores and on one core, and the cached decode step at batch 1 and 16 on all cores and on one
+    core.  Each is timed on one layer of its workload and scaled to the 64-layer stack."""
+    import oracle
+    f = oracle_layer_inputs()
+    cores = oracle.max_threads()
+    per_layer, reps = _timed_reps(lambda: oracle_step(f), min_seconds, max_reps)
     tok_s = PF["B"] * PF["L"] / (per_layer * PF["layers"])
-    return {"value": tok_s, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+    legs = {}
+    try:
+        oracle.set_threads(1)
+        t1, r1 = _timed_reps(lambda: oracle_step(f), 3.0, 3)
+        legs["prefill_1core"] = {"tokens_per_s": PF["B"] * PF["L"] / (t1 * PF["layers"]), "cores": 1,
+                                 "s_per_layer": t1, "runs": r1}
+        for bsz in (1, 16):
+            fd = oracle_decode_inputs(bsz)
+            for n_threads in (cores, 1):
+                oracle.set_threads(n_threads)
+                td, rd = _timed_reps(lambda: oracle_decode_layer(fd), 2.0, 200, min_reps=3)
+                legs[f"decode_b{bsz}_{'1core' if n_threads == 1 else 'all_cores'}"] = {
+                    "steps_per_s": 1.0 / (td * DEC["layers"]), "cores": n_threads, "s_per_layer": td,
+                    "runs": rd}
+    finally:
+        oracle.set_threads(cores)
+    return {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": (f"fp64 sequential recurrence on 1 of the 64 layers (all {PF['L']} tokens, "
-                       f"{PF['H']} heads), {len(times)} runs, median {per_layer:.3f} s per layer; "
-                       f"stack rate = per-layer rate / 64"),
+                       f"{PF['H']} heads), {reps} runs, median {per_layer:.3f} s per layer; "
+                       f"stack rate = per-layer rate / 64 (an extrapolation from one layer)"),
+            "legs": legs,
+            "legs_note": ("each leg times one layer of its workload and divides by 64 layers: prefill "
+                          "tokens/s of the 2.7B-shaped stack, decode steps/s of the 64-layer 2.7B-shaped "
+                          "cache at batch 1 and 16 (one fp64 decode step per layer)"),
             "host_cpu": _cpu_model(), "nproc": os.cpu_count()}
 
 
@@ -796,32 +850,46 @@ def main():
     flops_layer = prefill_flops(B, L, H, P, G, N, Q)
     tflops = flops_layer * PF["layers"] * world / (ms_step / 1e3) / 1e12
 
-    # roofline of the dominant kernel (largest summed device time)
+    # roofline of the dominant kernel (largest summed device time), in algorithmic work: its
+    # share of the method-level flops (the tensor-core kernels' target is a fraction of the
+    # bf16 tensor peak), else the method-level bytes it is responsible for against HBM
     kt = pf["kernel_times"]
     dom = max(kt, key=lambda n: kt[n][0])
     dms, dcnt = kt[dom]
     avg_s = dms / max(dcnt, 1) / 1e3
-    # Every tensor-core prefill kernel does far fewer flops per byte it must move than the
-    # measured ridge (~250 flop/B), so each is HBM-bound: achieved = its algorithmic bytes per
-    # launch / its event-timed average launch duration.
-    by = KERNEL_BYTES[dom](B, L, H, P, G, N)
-    ach = by / avg_s / 1e9
+    method_bytes = prefill_bytes(B, L, H, P, G, N)
     traffic = measured_traffic(dom)
-    roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "algorithmic_bytes": by,
-            "peak_source": f"{peaks['source']} copy", "avg_launch_us": avg_s * 1e6, "launches_timed": dcnt}
-    if dom in ("chunk_scan", "chunk_state"):
-        fl = (chunk_scan_flops if dom == "chunk_scan" else chunk_state_flops)(B, L, H, P, G, N, Q)
-        roof["tensor_tflops"] = fl / avg_s / 1e12
-        roof["tensor_frac"] = roof["tensor_tflops"] / peaks["bf16_tflops"]
+    if dom in KERNEL_METHOD_FLOPS:
+        fl = KERNEL_METHOD_FLOPS[dom](B, L, H, P, G, N, Q)
+        ach = fl / avg_s / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": traffic,
+                "algorithmic_flops": fl, "peak_source": f"{peaks['source']} bf16 matmul (burst)"}
+    else:
+        ach = method_bytes / avg_s / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "algorithmic_bytes": method_bytes,
+                "peak_source": f"{peaks['source']} copy"}
+    roof.update(avg_launch_us=avg_s * 1e6, launches_timed=dcnt)
+    # the whole layer against both roofs, and the DRAM bytes the kernels really move per layer
+    # (the ncu capture) over the method's own bytes
+    layer_s = ms_step / 1e3 / PF["layers"]
+    roof["method_frac_hbm"] = method_bytes / layer_s / 1e9 / peaks["hbm_gbs"]
+    roof["method_tensor_frac"] = flops_layer / layer_s / 1e12 / peaks["bf16_tflops"]
+    roof["method_bytes_per_layer"] = method_bytes
+    tr = [measured_traffic(n) for n in kt]
+    roof["traffic_ratio"] = sum(tr) / method_bytes if tr and all(t is not None for t in tr) else None
     kernels = {}
     for n, v in kt.items():
         avg = v[0] / max(v[1], 1) / 1e3
-        kb = KERNEL_BYTES[n](B, L, H, P, G, N) if n in KERNEL_BYTES else None
-        kernels[n] = {"total_ms": v[0], "launches": v[1], "avg_us": avg * 1e6}
-        if kb:
-            kernels[n].update(algorithmic_bytes=kb, gbs=kb / avg / 1e9, frac=kb / avg / 1e9 / peaks["hbm_gbs"],
-                              traffic=measured_traffic(n))
+        kernels[n] = {"total_ms": v[0], "launches": v[1], "avg_us": avg * 1e6, "traffic": measured_traffic(n)}
+        if n in KERNEL_BYTES:
+            mb = KERNEL_BYTES[n](B, L, H, P, G, N)
+            kernels[n].update(moved_bytes=mb, moved_gbs=mb / avg / 1e9, moved_frac=mb / avg / 1e9 / peaks["hbm_gbs"])
+        if n in KERNEL_METHOD_FLOPS:
+            fl = KERNEL_METHOD_FLOPS[n](B, L, H, P, G, N, Q)
+            kernels[n].update(method_flops=fl, tflops=fl / avg / 1e12,
+                              tensor_frac=fl / avg / 1e12 / peaks["bf16_tflops"])
 
     decode, by_context = {}, None
     if not args.no_decode:

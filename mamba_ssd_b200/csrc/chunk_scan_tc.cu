@@ -14,7 +14,9 @@
 //   CB  = C_k B_k^T                 once per (batch, block, group), kept in TMEM, fp32
 //   O   = C_k h_prev^T              h_prev^T arrives by TMA as a bf16 [n][p] tile
 //   P~  = mask(CB * dt_s * exp(acs_l - acs_s)) + D on the diagonal   (CUDA cores -> TMEM,
-//         from precomputed per-token factors colv = acs*log2(e) - log2(dt), acs2 = acs*log2(e))
+//         from precomputed per-token factors acs2 = acs*log2(e) and ldt = log2(dt); the
+//         exponent is (acs2_l - acs2_s) + ldt_s, the cumsums subtracted first so that ldt is
+//         not lost to rounding when the cumsum is large)
 //   Y   = P~ x_k                    A operand read from TMEM, x_k straight from its TMA tile
 //   y_l = Y_l + exp(acs_l) O_l      (epilogue, fp32 -> bf16)
 // Folding dt into the columns of P~ and D into its diagonal means x is used as loaded:
@@ -58,7 +60,7 @@ constexpr uint32_t kBox = R * 128;            // [128 rows][64 bf16] swizzled bo
 constexpr uint32_t kOffC = 0;                 // C block: 2 n-boxes, 32 KB
 constexpr uint32_t kOffB = 2 * kBox;          // B block: 2 n-boxes, 32 KB
 constexpr uint32_t kOffStage = 4 * kBox;      // ring of stages
-constexpr uint32_t kStX = 0, kStH = kBox, kStRows = 2 * kBox;  // x box, h_prev^T box, colv+acs2
+constexpr uint32_t kStX = 0, kStH = kBox, kStRows = 2 * kBox;  // x box, h_prev^T box, ldt+acs2
 constexpr uint32_t kStageBytes = 2 * kBox + 2048;             // keeps 1024-byte alignment
 constexpr uint32_t kOffOut = kOffStage + kStages * kStageBytes;  // y staging [128][64] bf16
 constexpr uint32_t kOffVb = kOffOut + kBox;                       // per-warp column factors
@@ -67,8 +69,8 @@ constexpr uint32_t kSmem = kOffBar + 256 + 1024;
 // TMEM columns: CB, then two sets of {P~ (bf16 pairs), Y, O}
 constexpr uint32_t kColCB = 0, kSet = 192, kSet0 = 128, kOffPT = 0, kOffY = 64, kOffO = 128;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kDiagFactorRange = 96.f;
-constexpr int kEpiBar = 1;  // named barrier of the epilogue warps  // log2 range of a diagonal sub-block that is factored
+constexpr float kDiagFactorRange = 96.f;  // log2 range of a diagonal sub-block that is factored
+constexpr int kEpiBar = 1;                 // named barrier of the epilogue warps
 }  // namespace csc
 
 __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
@@ -254,8 +256,8 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
             if (ok && j >= 2) ok = wait(&acc_full[t], ((j >> 1) - 1) & 1);
             if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform
             tc_fence_after();
-            const float *colv = reinterpret_cast<const float *>(stage(j) + kStRows);
-            const float *acs2 = colv + R;
+            const float *ldt = reinterpret_cast<const float *>(stage(j) + kStRows);
+            const float *acs2 = ldt + R;
             const float al = acs2[myrow];
             const uint32_t set = tmem + lane_base + kSet0 + t * kSet;
 #pragma unroll
@@ -268,9 +270,9 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
                 const bool diag = cb == rq;
                 const bool factored = !diag || acs2[cb * 32] - acs2[cb * 32 + 31] <= kDiagFactorRange;
                 if (factored) {
-                    // P~_ls = CB_ls * 2^(acs2_l - ref) * 2^(ref - colv_s); colv = acs2 - log2(dt)
+                    // P~_ls = CB_ls * 2^(acs2_l - ref) * 2^((ref - acs2_s) + ldt_s)
                     const float ref = diag ? acs2[cb * 32 + 15] : acs2[cb * 32 + 31];
-                    vb[lane] = ex2_approx(ref - colv[cb * 32 + lane]);
+                    vb[lane] = ex2_approx((ref - acs2[cb * 32 + lane]) + ldt[cb * 32 + lane]);
                     __syncwarp();
                     const float u = ex2_approx(al - ref);
                     tmem_wait_ld();
@@ -286,14 +288,15 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
                     __syncwarp();
                 } else {
                     tmem_wait_ld();
-                    const float4 *c4 = reinterpret_cast<const float4 *>(colv + cb * 32);
+                    const float4 *a4 = reinterpret_cast<const float4 *>(acs2 + cb * 32);
+                    const float4 *l4 = reinterpret_cast<const float4 *>(ldt + cb * 32);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const float4 c = c4[i];
-                        v[4 * i + 0] *= ex2_approx(al - c.x);
-                        v[4 * i + 1] *= ex2_approx(al - c.y);
-                        v[4 * i + 2] *= ex2_approx(al - c.z);
-                        v[4 * i + 3] *= ex2_approx(al - c.w);
+                        const float4 a = a4[i], l = l4[i];
+                        v[4 * i + 0] *= ex2_approx((al - a.x) + l.x);
+                        v[4 * i + 1] *= ex2_approx((al - a.y) + l.y);
+                        v[4 * i + 2] *= ex2_approx((al - a.z) + l.z);
+                        v[4 * i + 3] *= ex2_approx((al - a.w) + l.w);
                     }
                 }
                 if (diag) {  // causal mask and the D skip; a select, so what lies above is dropped

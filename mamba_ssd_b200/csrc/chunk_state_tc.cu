@@ -22,11 +22,13 @@
 //
 // The kernel also forms step a1 for the items it owns (the decay factors that the state pass
 // and the scan read): dt = clip(softplus(dt_raw + dt_bias)), A = -exp(A_log), the in-block
-// cumsum acs of dt*A, stored in log2 form as colv = acs*log2(e) - log2(dt) and
-// acs2 = acs*log2(e), so that dt_s exp(acs_l - acs_s) = exp2(acs2_l - colv_s).  Source: the
+// cumsum acs of dt*A, stored in log2 form as acs2 = acs*log2(e) and ldt = log2(dt), so that
+// dt_s exp(acs_l - acs_s) = exp2((acs2_l - acs2_s) + ldt_s).  The difference of the cumsums is
+// taken before log2(dt) is added: folded into one number, log2(dt) would be lost to rounding
+// once |acs2| is large (a decay of many nats per token).  Source: the
 // blog walk-through's §1.1 (discretisation, chunked cumulative decay) and §1.2 (the fused
 // softplus -> clip -> exp chain); §4.1 (the decay in float32).  Tokens past L get dt = 0, so
-// their decay is 1 and their weight exactly 0 (colv = +inf).
+// their decay is 1 and their weight exactly 0 (ldt = -inf).
 //
 // Structure: persistent CTAs, one per SM, each owning a contiguous range of (batch, block,
 // head) items (consecutive items share the block's B tile).  Warp-specialised:
@@ -57,7 +59,7 @@ constexpr int kStages = 4;
 constexpr int kThreads = (kPrepWarp + kStages) * 32;
 constexpr uint32_t kBox = R * 128;                 // [128 rows][64 bf16], 16 KB
 constexpr uint32_t kOffB = 0;                      // B block: 2 n-boxes, 32 KB
-constexpr uint32_t kStageBytes = 2 * kBox + 1024;  // x/hi box, lo box, colv[128] + acs2[128]
+constexpr uint32_t kStageBytes = 2 * kBox + 1024;  // x/hi box, lo box, ldt[128] + acs2[128]
 constexpr uint32_t kOffStage = 2 * kBox;
 constexpr uint32_t kOffOut = kOffStage + kStages * kStageBytes;  // S^T staging: 2 x [128][32] fp32
 constexpr uint32_t kOffBar = kOffOut + 2 * kBox;
@@ -236,14 +238,26 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
                 run += d[i] * A;
             }
             float acc = warp_inclusive_sum(run) - run;  // exclusive prefix of this lane
-            float cv[4], a2[4];
+            float lg[4], a2[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 acc += d[i] * A;
                 a2[i] = acc * kLog2e;
-                cv[i] = a2[i] - log2f(d[i]);
+                lg[i] = log2f(d[i]);
             }
-            const float4 c4 = make_float4(cv[0], cv[1], cv[2], cv[3]);
+            // a ragged last block: the padded slots take exactly the last real token's cumsum
+            // (the lanes' partial sums round differently; the block's end must stand for that
+            // token, so that its own weight exp2(acs2_end - acs2_last) is exactly 1)
+            const int tl = L - 1 - it.k * R;  // slot of the last real token
+            if (tl < R - 1) {                 // warp-uniform
+                const float mine = (tl >> 2) == lane ? ((tl & 3) == 0 ? a2[0] : (tl & 3) == 1 ? a2[1]
+                                                        : (tl & 3) == 2 ? a2[2] : a2[3]) : 0.f;
+                const float last = __shfl_sync(0xffffffffu, mine, tl >> 2);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (lane * 4 + i > tl) a2[i] = last;
+            }
+            const float4 c4 = make_float4(lg[0], lg[1], lg[2], lg[3]);
             const float4 a4 = make_float4(a2[0], a2[1], a2[2], a2[3]);
             float *rows = reinterpret_cast<float *>(stage(j) + 2 * kBox);
             reinterpret_cast<float4 *>(rows)[lane] = c4;
@@ -268,11 +282,12 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
             if (!__all_sync(0xffffffffu, wait(&st_full[s], (j / kStages) & 1))) break;  // warp-uniform
             uint8_t *xt = stage(j);
             uint8_t *lo = xt + kBox;
-            const float *colv = reinterpret_cast<const float *>(xt + 2 * kBox);
-            const float *acs2 = colv + R;
-            // w_s = dt_s exp(acs_last - acs_s) = exp2(acs2_last - colv_s); lanes 0..15 hold the
-            // weights of this warp's 16 rows
-            const float wl = lane < 16 ? ex2_approx(acs2[R - 1] - colv[tw * 16 + lane]) : 0.f;
+            const float *ldt = reinterpret_cast<const float *>(xt + 2 * kBox);
+            const float *acs2 = ldt + R;
+            // w_s = dt_s exp(acs_last - acs_s) = exp2((acs2_last - acs2_s) + ldt_s); lanes 0..15
+            // hold the weights of this warp's 16 rows
+            const int rw = tw * 16 + (lane & 15);
+            const float wl = lane < 16 ? ex2_approx((acs2[R - 1] - acs2[rw]) + ldt[rw]) : 0.f;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {  // 16 rows x 8 chunks = 128 chunks over 32 lanes
                 const int idx = q * 32 + lane;

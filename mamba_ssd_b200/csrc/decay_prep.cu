@@ -66,10 +66,23 @@ __global__ void __launch_bounds__(256) decay_prep_kernel(
         for (int i = 0; i < per; ++i) run += row[i] * A;
         float acc = warp_inclusive_sum(run) - run;  // exclusive prefix of this lane
         const size_t base = ((size_t)b * H + h) * Lp + (size_t)c * Q + lane * per;
+        // In a ragged last chunk the padded slots must hold exactly the cumsum of the last real
+        // token, the value the chunk's end stands for: the lanes' partial sums round
+        // differently, and exp(acs_end - acs_last) must be exactly 1, not exp(rounding) (which
+        // is far from 1, or infinite, when the cumsum is large).
+        const int tl = L - 1 - c * Q;  // slot of the last real token, when the chunk is ragged
+        const bool ragged = tl < Q - 1;
+        float last = 0.f;
         for (int i = 0; i < per; ++i) {
             acc += row[i] * A;
+            if (lane * per + i == tl) last = acc;
             acs[base + i] = acc;
             dtf[base + i] = row[i];
+        }
+        if (ragged) {  // warp-uniform
+            last = __shfl_sync(0xffffffffu, last, tl / per);
+            for (int i = 0; i < per; ++i)
+                if (lane * per + i > tl) acs[base + i] = last;
         }
     }
 }

@@ -47,7 +47,7 @@ cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t 
 // Prefill workspace layout, 256-byte aligned pieces:
 //   status int32 (256-byte slot): SSD_OK, or SSD_ERR_TIMEOUT if a bounded wait gave up
 //   dtf    [B][H][Lp]          clipped dt per token (0 past the end of the sequence); on the
-//                              tensor-core path colv = acs2 - log2(dt) instead
+//                              tensor-core path its base-2 logarithm, log2(dt), instead
 //   acs    [B][H][Lp]          inclusive cumsum of dt*A inside each block; on the tensor-core
 //                              path acs2 = that cumsum times log2(e)
 //   states [B][nb][H][P][N]    fp32 block states; the CUDA-core path overwrites them in
@@ -75,7 +75,7 @@ cudaError_t launch_decay_prep(int dtype, const void *dt, const float *A_log, con
 // tensor-core prefill (bf16 storage, P = 64, N = 128), 128-token blocks
 constexpr int kTcBlock = 128;
 bool prefill_tc_supported(int dtype, int P, int N);
-// chunk_state_tc also forms the log2-form decay factors (dtf = colv, acs = acs2) from dt and
+// chunk_state_tc also forms the log2-form decay factors (dtf = log2(dt), acs = acs2) from dt and
 // resets the status word: it is the first kernel of a tensor-core prefill call.
 cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
                                   const float *dt_bias, float dt_min, float dt_max, float *dtf, float *acs,

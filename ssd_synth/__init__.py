@@ -124,7 +124,7 @@ def _f32(a):
 # prefill inputs
 # ----------------------------------------------------------------------------------
 def prefill_inputs(B, L, H, P, G, N, dtype="bf16", seed=0, h0=False,
-                   dt_bias_zero=True, unclipped=False):
+                   dt_bias_zero=True, unclipped=False, a_log=None, dt_clip=None):
     """Seeded prefill inputs.
 
     Returns a dict whose entries are pairs (storage, f64) for
@@ -132,6 +132,9 @@ def prefill_inputs(B, L, H, P, G, N, dtype="bf16", seed=0, h0=False,
     storage dtype, and A_log[H], D[H], dt_bias[H], h0[B,H,P,N] (or None) in fp32,
     plus dt_min / dt_max.  ``unclipped`` widens the clip so the softplus branch is
     exercised over its whole range (the workload clip saturates ~60% of dt at 0.1).
+    ``a_log`` replaces the drawn A_log (a scalar for every head, or one value per head)
+    and ``dt_clip`` = (dt_min, dt_max) replaces the clip range: the decay edge cases
+    (no decay, full decay, steep decay inside one block) are made from these.
     """
     rng = np.random.default_rng(seed)
     x = rng.standard_normal((B, L, H, P), dtype=np.float32)
@@ -154,6 +157,10 @@ def prefill_inputs(B, L, H, P, G, N, dtype="bf16", seed=0, h0=False,
     }
     if unclipped:
         out["dt_min"], out["dt_max"] = 0.0, float("inf")
+    if a_log is not None:
+        out["A_log"] = _f32(np.broadcast_to(np.asarray(a_log, dtype=np.float32), (H,)).copy())
+    if dt_clip is not None:
+        out["dt_min"], out["dt_max"] = float(dt_clip[0]), float(dt_clip[1])
     if h0:
         out["h0"] = _f32(rng.standard_normal((B, H, P, N), dtype=np.float32)
                          * np.float32(math.sqrt(0.1)))

@@ -36,18 +36,22 @@ def test_tensor_core_kernel_bytes():
 
 
 def test_traffic_reported_only_for_the_captured_sources(tmp_path, monkeypatch):
-    rec = json.load(open(os.path.join(ROOT, bench.TRAFFIC_FILE)))
-    for name in bench.KERNEL_BYTES:
-        assert bench.measured_traffic(name) == rec[name]["dram_bytes"]
-    assert bench.measured_traffic("no_such_kernel") is None
-    # a record whose hash does not match the sources is not reported
-    stale = {k: dict(v, source_sha256="0" * 64) for k, v in rec.items()}
+    # a record taken with the current sources is reported; one whose hash does not match the
+    # sources (the kernel changed since the capture) is not
+    names = list(bench.KERNEL_SOURCES)
+    fresh = {n: {"dram_bytes": 1e6 * (i + 1), "source_sha256": bench.kernel_source_sha(n)}
+             for i, n in enumerate(names)}
     fake_root = tmp_path / "repo"
     (fake_root / "profiles").mkdir(parents=True)
-    (fake_root / bench.TRAFFIC_FILE).write_text(json.dumps(stale))
+    (fake_root / bench.TRAFFIC_FILE).write_text(json.dumps(fresh))
     monkeypatch.setattr(bench, "ROOT", str(fake_root))
+    # the sources are hashed under the real root, before ROOT pointed at the fake one
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda name: fresh[name]["source_sha256"])
+    for i, name in enumerate(names):
+        assert bench.measured_traffic(name) == 1e6 * (i + 1)
+    assert bench.measured_traffic("no_such_kernel") is None
     monkeypatch.setattr(bench, "kernel_source_sha", lambda name: "1" * 64)
-    for name in bench.KERNEL_BYTES:
+    for name in names:
         assert bench.measured_traffic(name) is None
 
 

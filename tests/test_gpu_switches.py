@@ -34,3 +34,9 @@ def test_without_programmatic_dependent_launch():
 def test_cuda_core_path_on_tensor_core_shapes():
     run_child({"SSD_PREFILL_KERNELS": "simt"},
               [os.path.join(HERE, "test_gpu_prefill.py"), "-k", "m130m or m1p3b_b8 or sweep"])
+
+
+def test_cuda_core_path_on_decay_edge_cases():
+    # no decay, full decay and steep in-block decay on the float32 CUDA-core kernels, for the
+    # bf16 shapes that otherwise run on the tensor cores
+    run_child({"SSD_PREFILL_KERNELS": "simt"}, [os.path.join(HERE, "test_gpu_decay_edges.py")])
