@@ -107,17 +107,48 @@ def chunk_scan_bytes(B, L, H, P, G, N, e=2):
     return B * L * (2 * H * P * e + 2 * G * N * e) + B * nk * H * N * P * 2 + 2 * B * H * nk * TC_BLOCK * 4
 
 
-KERNEL_BYTES = {"chunk_state": chunk_state_bytes, "state_pass": state_pass_bytes, "chunk_scan": chunk_scan_bytes}
+# The fused tensor-core prefill (the default for these shapes): work in units of (head pair,
+# 128-token block), CTA ranges cut into runs per head pair; each run leaves one [N][P] fp32
+# state per head in a slot (chains + CTAs slots at most).
+N_SMS = 148
+
+
+def _run_slots(B, L, H):
+    nch = B * (H // 2)
+    return (nch + min(nch * _tc_blocks(L), N_SMS)) * 2  # one state per head of each slot
+
+
+def run_state_bytes(B, L, H, P, G, N, e=2):
+    """x, B, dt in; each run's state (and its decay) out."""
+    return B * L * (H * P * e + G * N * e + H * e) + _run_slots(B, L, H) * (N * P * 4 + 4)
+
+
+def run_pass_bytes(B, L, H, P, G, N, h0=False):
+    """The run states read and overwritten by the carry-ins; h_final (and h0)."""
+    return 2 * _run_slots(B, L, H) * N * P * 4 + (2 if h0 else 1) * B * H * P * N * 4
+
+
+def chunk_scan_fused_bytes(B, L, H, P, G, N, e=2):
+    """x, B, C, dt and the carry-ins in; y out."""
+    return B * L * (2 * H * P * e + 2 * G * N * e + H * e) + _run_slots(B, L, H) * N * P * 4
+
+
+KERNEL_BYTES = {"chunk_state": chunk_state_bytes, "state_pass": state_pass_bytes, "chunk_scan": chunk_scan_bytes,
+                "run_state": run_state_bytes, "run_pass": run_pass_bytes, "chunk_scan_fused": chunk_scan_fused_bytes}
 # Each kernel's share of the method-level flops (the dense-tile count of prefill_flops at the
 # caller's chunk): the block state is step a3 (2HNP per token), the chunk scan steps a2 + a5 (CB once
 # per group, the masked product, C h_prev); the state pass is step a4, a scan with no
 # contraction.
-KERNEL_METHOD_FLOPS = {"chunk_state": chunk_state_flops, "chunk_scan": chunk_scan_flops}
+KERNEL_METHOD_FLOPS = {"chunk_state": chunk_state_flops, "chunk_scan": chunk_scan_flops,
+                       "run_state": chunk_state_flops, "chunk_scan_fused": chunk_scan_flops}
 # The sources a kernel's DRAM-traffic capture depends on: a capture is used only while these
 # files are byte-identical to the ones it was taken with.
-KERNEL_SOURCES = {"chunk_state": ["chunk_state_tc.cu"], "state_pass": ["state_pass.cu"],
-                  "chunk_scan": ["chunk_scan_tc.cu"]}
-SHARED_SOURCES = ["common.cuh", "tc.cuh", "items.cuh", "launch.h", "tmap.cu"]
+KERNEL_SOURCES = {"chunk_state": ["chunk_state_tc.cu", "items.cuh"], "state_pass": ["state_pass.cu"],
+                  "chunk_scan": ["chunk_scan_tc.cu", "items.cuh"], "run_state": ["run_state_tc.cu", "runs.cuh"],
+                  "run_pass": ["run_pass.cu", "runs.cuh"], "chunk_scan_fused": ["chunk_scan_fused.cu", "runs.cuh"]}
+SHARED_SOURCES = ["common.cuh", "tc.cuh", "launch.h", "tmap.cu"]
+PREFILL_KERNELS = ["decay_prep", "chunk_state", "state_pass", "chunk_scan", "run_state", "run_pass",
+                   "chunk_scan_fused"]
 TRAFFIC_FILE = os.path.join("profiles", "prefill_traffic_m2p7b_layer.json")
 
 
@@ -480,10 +511,9 @@ def bench_prefill(args, torch, ssd, device, rank, world):
     ms = start.elapsed_time(end)
     ms_max = max_over_ranks(ms, world, device)
 
-    names = ["decay_prep", "chunk_state", "state_pass", "chunk_scan"]
     with torch.cuda.stream(stream):
-        kt = kernel_times(torch, lib, step_eager, names)
-    kt = {n: v for n, v in kt.items() if v[1] > 0}  # the tensor-core path has no separate decay kernel
+        kt = kernel_times(torch, lib, step_eager, PREFILL_KERNELS)
+    kt = {n: v for n, v in kt.items() if v[1] > 0}  # only the kernels of the path that ran
     del graph
     return dict(ms_total=ms_max, launches_per_step=launches_per_step, kernel_times=kt,
                 clocks=clocks.summary())

@@ -18,8 +18,22 @@ thread_local int g_last_cuda_error = 0;
 
 // ---- profiling hooks: launch counter and optional per-kernel CUDA-event timing ----
 const char *const kKernelNames[] = {"decay_prep",  "chunk_state",   "state_pass",  "chunk_scan",
-                                    "decode_step", "causal_conv1d", "decode_conv", "gated_rmsnorm"};
-enum KernelId { K_DECAY = 0, K_STATE, K_PASS, K_SCAN, K_DECODE, K_CONV, K_DCONV, K_NORM, K_COUNT };
+                                    "decode_step", "causal_conv1d", "decode_conv", "gated_rmsnorm",
+                                    "run_state",   "run_pass",      "chunk_scan_fused"};
+enum KernelId {
+    K_DECAY = 0,
+    K_STATE,
+    K_PASS,
+    K_SCAN,
+    K_DECODE,
+    K_CONV,
+    K_DCONV,
+    K_NORM,
+    K_RSTATE,
+    K_RPASS,
+    K_FSCAN,
+    K_COUNT
+};
 
 std::atomic<long long> g_launches{0};
 std::atomic<int> g_timer_on{0};
@@ -86,13 +100,27 @@ bool pdl_enabled() {
 
 namespace {
 // Tensor-core kernels are used wherever they apply, unless SSD_PREFILL_KERNELS=simt is set in
-// the environment (then every shape runs on the float32 CUDA-core kernels).
+// the environment (then every shape runs on the float32 CUDA-core kernels).  By default the
+// tensor-core path is the block-state one (per-block states through memory, one state pass);
+// SSD_PREFILL_KERNELS=fused selects the run-carrying kernels for the shapes they support
+// (each head pair's state carried through runs of blocks on chip: a fraction of the memory
+// traffic, but slower on B200 as measured, so not the default).
 bool use_tensor_cores() {
     static const bool on = [] {
         const char *v = getenv("SSD_PREFILL_KERNELS");
         return !(v && strcmp(v, "simt") == 0);
     }();
     return on;
+}
+bool use_fused() {
+    static const bool on = [] {
+        const char *v = getenv("SSD_PREFILL_KERNELS");
+        return v && strcmp(v, "fused") == 0;
+    }();
+    return on;
+}
+bool fused_path(int dtype, int L, int P, int N, int H, int G) {
+    return L > 0 && use_fused() && ssd::prefill_fused_supported(dtype, P, N, H, G);
 }
 
 int sm_count() {
@@ -150,18 +178,50 @@ PrefillWorkspace carve_prefill_workspace(void *base, int B, int L, int H, int P,
     return w;
 }
 
-// Bytes a prefill needs: the larger of the layouts its shape may run with, so that a
-// workspace sized by the query serves either path.
-size_t prefill_query_bytes(int B, int L, int H, int P, int N, int chunk, int dtype) {
-    size_t need = prefill_workspace_bytes(B, L, H, P, N, chunk, false);
-    if (prefill_tc_supported(dtype, P, N)) {
-        const size_t tc = prefill_workspace_bytes(B, L, H, P, N, kTcBlock, true);
+RunLayout fused_layout(int B, int L, int H, int num_sms) {
+    RunLayout lay;
+    lay.nk = cdiv(L, kTcBlock);
+    lay.nch = B * (H / kPairHeads);
+    lay.U = lay.nch * lay.nk;
+    int g = num_sms < kMaxCtas ? num_sms : kMaxCtas;
+    lay.grid = lay.U < g ? lay.U : g;
+    return lay;
+}
+
+// sized for the largest grid the kernels may use (kMaxCtas), whatever the device
+size_t fused_workspace_bytes(int B, int L, int H) {
+    const RunLayout lay = fused_layout(B, L, H, kMaxCtas);
+    const size_t slots = (size_t)lay.slots() * kPairHeads;
+    return kStatusSlot + align_up(slots * 128 * 64 * sizeof(float), 256) + align_up(slots * sizeof(float), 256);
+}
+
+FusedWorkspace carve_fused_workspace(void *base, int B, int L, int H) {
+    const RunLayout lay = fused_layout(B, L, H, kMaxCtas);
+    const size_t slots = (size_t)lay.slots() * kPairHeads;
+    char *p = static_cast<char *>(base);
+    FusedWorkspace w;
+    w.status = reinterpret_cast<int *>(p);
+    w.slots = reinterpret_cast<float *>(p + kStatusSlot);
+    w.decays = reinterpret_cast<float *>(p + kStatusSlot + align_up(slots * 128 * 64 * sizeof(float), 256));
+    return w;
+}
+
+}  // namespace ssd
+
+namespace {
+// Bytes a prefill needs on the path its shape runs (the environment switches, read once per
+// process, decide the path the same way for the query and the call).
+size_t prefill_query_bytes(int B, int L, int H, int P, int G, int N, int chunk, int dtype) {
+    if (fused_path(dtype, L, P, N, H, G)) return ssd::fused_workspace_bytes(B, L, H);
+    size_t need = ssd::prefill_workspace_bytes(B, L, H, P, N, chunk, false);
+    if (use_tensor_cores() && ssd::prefill_tc_supported(dtype, P, N)) {
+        const size_t tc = ssd::prefill_workspace_bytes(B, L, H, P, N, ssd::kTcBlock, true);
         if (tc > need) need = tc;
     }
     return need;
 }
 
-}  // namespace ssd
+}  // namespace
 
 extern "C" {
 
@@ -185,7 +245,7 @@ size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, int N, i
                                      int dtype) {
     if (check_prefill_shape(B, L, H, P, G, N, chunk, dtype) != SSD_OK) return 0;
     if (B == 0) return 0;
-    return ssd::prefill_query_bytes(B, L, H, P, N, chunk, dtype);
+    return prefill_query_bytes(B, L, H, P, G, N, chunk, dtype);
 }
 
 int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const void *Bm,
@@ -205,11 +265,29 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
         if (!aligned16(x) || !aligned16(dt) || !aligned16(Bm) || !aligned16(Cm) || !aligned16(y))
             return SSD_ERR_INVALID_ARG;
     }
-    const size_t need = ssd::prefill_query_bytes(B, L, H, P, N, chunk, dtype);
+    const size_t need = prefill_query_bytes(B, L, H, P, G, N, chunk, dtype);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return SSD_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
+    if (fused_path(dtype, L, P, N, H, G)) {
+        // fused tensor-core path: run states, the pass over runs, the scan carrying the states
+        const ssd::RunLayout lay = ssd::fused_layout(B, L, H, sm_count());
+        ssd::FusedWorkspace ws = ssd::carve_fused_workspace(workspace, B, L, H);
+        e = timed_launch(K_RSTATE, st, [&] {
+            return ssd::launch_run_state_tc(x, Bm, dt, A_log, dt_bias, dt_min, dt_max, ws.slots, ws.decays,
+                                            ws.status, B, L, H, G, lay, st);
+        });
+        if (e != cudaSuccess) return cuda_status(e);
+        e = timed_launch(K_RPASS, st,
+                         [&] { return ssd::launch_run_pass(ws.slots, ws.decays, h0, h_final, B, H, lay, st); });
+        if (e != cudaSuccess) return cuda_status(e);
+        e = timed_launch(K_FSCAN, st, [&] {
+            return ssd::launch_chunk_scan_fused(x, Bm, Cm, dt, A_log, dt_bias, dt_min, dt_max, D, ws.slots, y,
+                                                ws.status, B, L, H, G, lay, st);
+        });
+        return cuda_status(e);
+    }
     if (use_tensor_cores() && ssd::prefill_tc_supported(dtype, P, N)) {
         // tensor-core path: 128-token blocks, block states in fp32, h_prev^T in bf16
         const int blk = ssd::kTcBlock;
@@ -293,7 +371,7 @@ int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float *A_log,
     for (int i = 0; i < n_seq; ++i)
         if (((size_t)cu_seqlens[i] * H * e) % 16 != 0 || ((size_t)cu_seqlens[i] * G * N * e) % 16 != 0)
             return SSD_ERR_UNSUPPORTED;
-    const size_t need = ssd::prefill_query_bytes(1, max_len, H, P, N, chunk, dtype);
+    const size_t need = prefill_query_bytes(1, max_len, H, P, G, N, chunk, dtype);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return SSD_ERR_WORKSPACE;
     // every argument is valid: run each sequence through the prefill, in order on the stream,

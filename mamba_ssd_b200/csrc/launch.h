@@ -7,6 +7,8 @@
 
 #include <atomic>
 
+#include "runs.cuh"
+
 namespace ssd {
 
 // A kernel's dynamic shared-memory limit, raised once per device (the attribute is per device;
@@ -88,6 +90,34 @@ cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, 
 cudaError_t launch_state_pass_t(const float *states, const float *acs, const float *h0, float *h_final,
                                 __nv_bfloat16 *hT, int B, int L, int H, int P, int N, int chunk,
                                 cudaStream_t st);
+
+// Fused tensor-core prefill (bf16 storage, P = 64, N = 128, an even number of heads per
+// group): the work is split into runs of blocks per head pair (runs.cuh); three launches:
+//   run_state_tc      each run's own state (hi/lo accurate) and total decay, into its slot;
+//                     resets the status word (the first kernel of the call)
+//   run_pass          the pass over each chain's runs: carry-ins in place of the run states,
+//                     and h_final
+//   chunk_scan_fused  y, with each head's state carried through its runs in TMEM
+// Workspace: status (256-byte slot), then slots [lay.slots()][2][N][P] fp32, then decays
+// [lay.slots()][2] fp32 (log2 of each run's total decay), each piece 256-byte aligned.
+bool prefill_fused_supported(int dtype, int P, int N, int H, int G);
+struct FusedWorkspace {
+    int *status;
+    float *slots;
+    float *decays;
+};
+RunLayout fused_layout(int B, int L, int H, int num_sms);
+size_t fused_workspace_bytes(int B, int L, int H);
+FusedWorkspace carve_fused_workspace(void *base, int B, int L, int H);
+cudaError_t launch_run_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
+                                const float *dt_bias, float dt_min, float dt_max, float *slots, float *decays,
+                                int *status, int B, int L, int H, int G, const RunLayout &lay, cudaStream_t st);
+cudaError_t launch_run_pass(float *slots, const float *decays, const float *h0, float *h_final, int B, int H,
+                            const RunLayout &lay, cudaStream_t st);
+cudaError_t launch_chunk_scan_fused(const void *x, const void *Bm, const void *Cm, const void *dt, const float *A_log,
+                                    const float *dt_bias, float dt_min, float dt_max, const float *D,
+                                    const float *slots, void *y, int *status, int B, int L, int H, int G,
+                                    const RunLayout &lay, cudaStream_t st);
 
 cudaError_t launch_chunk_state(int dtype, const void *x, const void *Bm, const float *dtf,
                                const float *acs, float *states, int B, int L, int H, int G, int N,

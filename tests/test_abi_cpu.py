@@ -5,6 +5,8 @@ import ctypes
 import glob
 import os
 import re
+import subprocess
+import sys
 
 import pytest
 
@@ -50,9 +52,24 @@ def _layout(B, Lx, H, P, N, block, transposed):
     return 256 + 2 * per_tok + states + hT
 
 
-def ws_bytes(B, Lx, H, P, N, chunk, tensor_core_shape):
-    """The larger of the CUDA-core layout (caller's chunk) and, for bf16 P=64 N=128, the
-    tensor-core layout (128-token blocks plus a bf16 copy of the carried states)."""
+def _fused_layout(B, Lx, H):
+    """Status slot, then the run slots (one [N][P] fp32 state per head of a head pair) and the
+    runs' decays: chains = B * H / 2, units = chains * ceil(L / 128), slots = chains + the
+    largest grid (min(units, 160))."""
+    up = lambda v: -(-v // 256) * 256
+    nch = B * (H // 2)
+    units = nch * -(-Lx // 128)
+    slots = (nch + min(units, 160)) * 2
+    return 256 + up(slots * 128 * 64 * 4) + up(slots * 4)
+
+
+def ws_bytes(B, Lx, H, P, G, N, chunk, tensor_core_shape, fused=False):
+    """With the fused kernels selected (SSD_PREFILL_KERNELS=fused), bf16 P=64 N=128 with an even
+    number of heads per group and L > 0 needs only their run slots.  Otherwise: the larger of
+    the CUDA-core layout (caller's chunk) and, for bf16 P=64 N=128, the block-state tensor-core
+    layout (128-token blocks plus a bf16 copy of the carried states)."""
+    if fused and tensor_core_shape and Lx > 0 and (H // G) % 2 == 0:
+        return _fused_layout(B, Lx, H)
     need = _layout(B, Lx, H, P, N, chunk, False)
     if tensor_core_shape:
         need = max(need, _layout(B, Lx, H, P, N, 128, True))
@@ -61,15 +78,29 @@ def ws_bytes(B, Lx, H, P, N, chunk, tensor_core_shape):
 
 @pytest.mark.parametrize("shape", [(1, 4096, 80, 64, 1, 128, 256), (8, 2048, 64, 64, 1, 128, 256),
                                    (2, 300, 4, 64, 2, 16, 64), (1, 1, 4, 64, 1, 32, 128),
-                                   (1, 0, 4, 64, 1, 16, 256)])
+                                   (1, 0, 4, 64, 1, 16, 256), (1, 300, 6, 64, 2, 128, 256),
+                                   (1, 0, 8, 64, 1, 128, 256)])
 def test_prefill_workspace_size(shape):
     B, Lx, H, P, G, N, chunk = shape
     got = L.ssd_chunk_scan_workspace_size(B, Lx, H, P, G, N, chunk, BF16)
-    assert got == ws_bytes(B, Lx, H, P, N, chunk, P == 64 and N == 128) and got % 256 == 0
+    assert got == ws_bytes(B, Lx, H, P, G, N, chunk, P == 64 and N == 128) and got % 256 == 0
     got32 = L.ssd_chunk_scan_workspace_size(B, Lx, H, P, G, N, chunk, F32)
-    assert got32 == ws_bytes(B, Lx, H, P, N, chunk, False)
+    assert got32 == ws_bytes(B, Lx, H, P, G, N, chunk, False)
     assert L.ssd_chunk_scan_workspace_size(0, Lx, H, P, G, N, chunk, BF16) == 0
     assert L.ssd_chunk_scan_workspace_size(B, Lx, H, 32, G, N, chunk, BF16) == 0   # unsupported P
+
+
+@pytest.mark.parametrize("shape", [(1, 4096, 80, 64, 1, 128, 256), (8, 2048, 64, 64, 1, 128, 256),
+                                   (1, 300, 6, 64, 2, 128, 256), (1, 0, 8, 64, 1, 128, 256)])
+def test_prefill_workspace_size_fused(shape):
+    # the environment switch is read once per process: query it in a child
+    B, Lx, H, P, G, N, chunk = shape
+    code = ("import sys; sys.path.insert(0, %r); from mamba_ssd_b200 import _lib; "
+            "print(_lib.lib().ssd_chunk_scan_workspace_size(%d, %d, %d, %d, %d, %d, %d, 1))"
+            % (ROOT, B, Lx, H, P, G, N, chunk))
+    env = dict(os.environ, SSD_PREFILL_KERNELS="fused")
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, check=True)
+    assert int(out.stdout.strip()) == ws_bytes(B, Lx, H, P, G, N, chunk, True, fused=True)
 
 
 def prefill(**kw):

@@ -4,7 +4,11 @@ child process over a subset of the parity tests:
   SSD_PDL=0                    the tensor-core prefill and the decode step launched as
                                ordinary kernels (no programmatic dependent launch);
   SSD_PREFILL_KERNELS=simt     every prefill on the float32 CUDA-core kernels, including the
-                               bf16 P = 64, N = 128 shapes that otherwise use the tensor cores.
+                               bf16 P = 64, N = 128 shapes that otherwise use the tensor cores;
+  SSD_PREFILL_KERNELS=fused    the run-carrying tensor-core kernels (run states, the pass over
+                               runs, the scan carrying each head pair's state on chip) for the
+                               shapes they take: the prefill, decay-edge, graph and varlen
+                               parity suites run on them.
 """
 import os
 import subprocess
@@ -40,3 +44,10 @@ def test_cuda_core_path_on_decay_edge_cases():
     # no decay, full decay and steep in-block decay on the float32 CUDA-core kernels, for the
     # bf16 shapes that otherwise run on the tensor cores
     run_child({"SSD_PREFILL_KERNELS": "simt"}, [os.path.join(HERE, "test_gpu_decay_edges.py")])
+
+
+def test_fused_run_kernels():
+    run_child({"SSD_PREFILL_KERNELS": "fused"},
+              [os.path.join(HERE, "test_gpu_prefill.py"), os.path.join(HERE, "test_gpu_decay_edges.py"),
+               os.path.join(HERE, "test_gpu_varlen.py"), os.path.join(HERE, "test_gpu_graph.py"),
+               "-k", "not decode"])

@@ -45,7 +45,9 @@ def test_noalloc_matches_workspace_entry_twice(dtype, B, L, H, N, chunk, h0):
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
-    B, L, H, P, G, N, chunk = 1, 4096, 80, 64, 1, 128, 256  # a 2.7B-shaped layer needs 128.5 MB
+    # 16 sequences of the 2.7B head count: beyond the 48 MiB scratch on either tensor-core path
+    # (128 MB of block states, or 52.4 MB of run states with the fused kernels)
+    B, L, H, P, G, N, chunk = 16, 256, 80, 64, 1, 128, 256
     need = _lib.lib().ssd_chunk_scan_workspace_size(B, L, H, P, G, N, chunk, _lib.SSD_DTYPE_BF16)
     assert need > _lib.SSD_NOALLOC_SCRATCH_BYTES
     x = torch.empty((B, L, H, P), device="cuda", dtype=torch.bfloat16)
