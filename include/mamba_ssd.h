@@ -145,6 +145,9 @@ SSD_API int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log
  * SSD_ERR_UNSUPPORTED for a shape ssd_chunk_scan_fwd would not take or a sequence whose dt
  * rows would not start 16-byte aligned (never when H * sizeof(element) is a multiple of 16),
  * SSD_ERR_WORKSPACE.  A CUDA launch error stops the loop and is returned as SSD_ERR_CUDA.
+ * The workspace's status word is reset once for the whole call (a 4-byte memset on `stream`)
+ * and kept across the sequences: ssd_chunk_scan_status then reports SSD_ERR_TIMEOUT if any
+ * sequence's bounded waits gave up.
  */
 SSD_API int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float *A_log, const void *Bm,
                                       const void *Cm, const float *D, const float *dt_bias, float dt_min,
@@ -156,7 +159,11 @@ SSD_API int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float
  * Diagnostic: waits for `stream` to finish (this call synchronises, unlike every other
  * entry point) and returns the status the last ssd_chunk_scan_fwd on `workspace` left
  * there: SSD_OK, or SSD_ERR_TIMEOUT if one of its bounded device-side waits gave up (its
- * outputs are then incomplete).  SSD_ERR_CUDA if the stream or the copy failed.
+ * outputs are then incomplete).  A NULL workspace reads the built-in scratch of
+ * ssd_chunk_scan_fwd_noalloc on the current device, i.e. the status of the last
+ * allocation-free call there.  For ssd_chunk_scan_varlen_fwd it is the status of the whole
+ * call: SSD_ERR_TIMEOUT if any sequence's kernels timed out.  SSD_ERR_CUDA if the stream,
+ * the copy or the scratch lookup failed.
  */
 SSD_API int ssd_chunk_scan_status(const void *workspace, void *stream);
 
@@ -172,19 +179,26 @@ SSD_API int ssd_chunk_scan_status(const void *workspace, void *stream);
  *
  * What it does: exactly ssd_chunk_scan_fwd (same arguments, same kernels, same results),
  * except that the scratch comes from one device array of SSD_NOALLOC_SCRATCH_BYTES compiled
- * into this library instead of a caller-provided workspace.  Every GPU that loads the
- * library holds that array until the process exits.  Inputs and outputs are still the
- * caller's.
+ * into this library instead of a caller-provided workspace.  Every GPU on which the
+ * library's device code is loaded holds that array until the process exits (see the lazy
+ * loading note below for when that happens).  Inputs and outputs are still the caller's.
  *   - Shapes whose ssd_chunk_scan_workspace_size exceeds SSD_NOALLOC_SCRATCH_BYTES return
  *     SSD_ERR_WORKSPACE without launching anything (48 MiB covers, for example, one
  *     130M-shaped layer: batch 1, L = 4096, H = 24, P = 64, N = 128, bf16).
- *   - The first call on each device looks up the array's device address on that device (the
- *     device must be current); make that first call before any stream capture.
+ *   - Every call looks up the array's device address on the current device (cheap once the
+ *     library is loaded there; right across a device reset).  With lazy module loading, the
+ *     CUDA default, the first call on a device also loads the library's device code there,
+ *     and that is when the array's 48 MiB are committed on that device: make that first call
+ *     at start-up, before any stream capture and before an engine reserves the rest of the
+ *     device memory.  Later calls allocate nothing.
+ *   - Its status word (SSD_ERR_TIMEOUT if a bounded device-side wait gave up) is read with
+ *     ssd_chunk_scan_status(NULL, stream).
  *   - Every call uses the same array and leaves its contents behind.  Calls that may overlap
  *     on the GPU (different streams, different host threads without ordering) race on it and
  *     corrupt each other's results; order them on one stream.  Nothing in the array has to be
  *     zeroed by the caller.
- *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine; the one commit of the
+ *     array's memory is the driver's, when it loads the library's device code (above).
  */
 #define SSD_NOALLOC_SCRATCH_BYTES (48u * 1024u * 1024u)
 SSD_API int ssd_chunk_scan_fwd_noalloc(const void *x, const void *dt, const float *A_log,

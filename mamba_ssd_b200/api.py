@@ -158,7 +158,9 @@ def ssd_chunk_scan_fwd_noalloc(x, dt, A_log, Bm, Cm, D=None, chunk=256, h0=None,
 
 def ssd_chunk_scan_status(workspace, stream=None):
     """Synchronises the stream and returns the status word the last prefill on `workspace`
-    left: SSD_OK (0), or SSD_ERR_TIMEOUT (5) if a bounded wait in a kernel gave up."""
+    left: SSD_OK (0), or SSD_ERR_TIMEOUT (5) if a bounded wait in a kernel gave up.
+    workspace=None reads the built-in scratch of ssd_chunk_scan_fwd_noalloc on the current
+    device."""
     return _lib.lib().ssd_chunk_scan_status(_ptr(workspace), _stream(stream))
 
 

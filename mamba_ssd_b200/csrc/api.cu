@@ -248,11 +248,15 @@ size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, int N, i
     return prefill_query_bytes(B, L, H, P, G, N, chunk, dtype);
 }
 
-int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const void *Bm,
-                       const void *Cm, const float *D, const float *dt_bias, float dt_min,
-                       float dt_max, const float *h0, void *y, float *h_final, int B, int L,
-                       int H, int P, int G, int N, int chunk, int dtype, void *workspace,
-                       size_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+// The prefill.  reset_status: the call's first kernel resets the workspace status word (a
+// single call); the varlen prefill resets it once itself and keeps it across its sequences.
+int prefill(const void *x, const void *dt, const float *A_log, const void *Bm, const void *Cm, const float *D,
+            const float *dt_bias, float dt_min, float dt_max, const float *h0, void *y, float *h_final, int B, int L,
+            int H, int P, int G, int N, int chunk, int dtype, void *workspace, size_t workspace_bytes, void *stream,
+            bool reset_status) {
     int s = check_prefill_shape(B, L, H, P, G, N, chunk, dtype);
     if (s != SSD_OK) return s;
     if ((s = check_dt_range(dt_min, dt_max)) != SSD_OK) return s;
@@ -276,7 +280,7 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
         ssd::FusedWorkspace ws = ssd::carve_fused_workspace(workspace, B, L, H);
         e = timed_launch(K_RSTATE, st, [&] {
             return ssd::launch_run_state_tc(x, Bm, dt, A_log, dt_bias, dt_min, dt_max, ws.slots, ws.decays,
-                                            ws.status, B, L, H, G, lay, st);
+                                            ws.status, reset_status, B, L, H, G, lay, st);
         });
         if (e != cudaSuccess) return cuda_status(e);
         e = timed_launch(K_RPASS, st,
@@ -296,7 +300,7 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
             // the state kernel also forms the decay factors (step a1) of the items it owns
             e = timed_launch(K_STATE, st, [&] {
                 return ssd::launch_chunk_state_tc(x, Bm, dt, A_log, dt_bias, dt_min, dt_max, ws.dtf, ws.acs,
-                                                  ws.states, ws.status, B, L, H, G, sm_count(), st);
+                                                  ws.states, ws.status, reset_status, B, L, H, G, sm_count(), st);
             });
             if (e != cudaSuccess) return cuda_status(e);
         }
@@ -318,7 +322,7 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
     if (L > 0) {
         e = timed_launch(K_DECAY, st, [&] {
             return ssd::launch_decay_prep(dtype, dt, A_log, dt_bias, dt_min, dt_max, ws.dtf, ws.acs,
-                                          ws.status, B, L, H, chunk, st);
+                                          reset_status ? ws.status : nullptr, B, L, H, chunk, st);
         });
         if (e != cudaSuccess) return cuda_status(e);
         e = timed_launch(K_STATE, st, [&] {
@@ -338,6 +342,18 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
         if (e != cudaSuccess) return cuda_status(e);
     }
     return SSD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const void *Bm, const void *Cm,
+                       const float *D, const float *dt_bias, float dt_min, float dt_max, const float *h0, void *y,
+                       float *h_final, int B, int L, int H, int P, int G, int N, int chunk, int dtype,
+                       void *workspace, size_t workspace_bytes, void *stream) {
+    return prefill(x, dt, A_log, Bm, Cm, D, dt_bias, dt_min, dt_max, h0, y, h_final, B, L, H, P, G, N, chunk,
+                   dtype, workspace, workspace_bytes, stream, true);
 }
 
 int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float *A_log, const void *Bm,
@@ -375,7 +391,11 @@ int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float *A_log,
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return SSD_ERR_WORKSPACE;
     // every argument is valid: run each sequence through the prefill, in order on the stream,
-    // sharing the workspace (each call's kernels start after the previous call's have ended)
+    // sharing the workspace (each call's kernels start after the previous call's have ended).
+    // The status word is reset once here and kept across the sequences, so that a timeout in
+    // any of them is what ssd_chunk_scan_status reports for the call.
+    cudaError_t e0 = cudaMemsetAsync(workspace, 0, sizeof(int), static_cast<cudaStream_t>(stream));
+    if (e0 != cudaSuccess) return cuda_status(e0);
     const size_t state = (size_t)H * P * N;
     for (int i = 0; i < n_seq; ++i) {
         const size_t t0 = (size_t)cu_seqlens[i];
@@ -383,18 +403,23 @@ int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float *A_log,
         const char *xb = static_cast<const char *>(x), *dtb = static_cast<const char *>(dt);
         const char *bb = static_cast<const char *>(Bm), *cb = static_cast<const char *>(Cm);
         char *yb = static_cast<char *>(y);
-        s = ssd_chunk_scan_fwd(xb ? xb + t0 * H * P * e : nullptr, dtb ? dtb + t0 * H * e : nullptr, A_log,
-                               bb ? bb + t0 * G * N * e : nullptr, cb ? cb + t0 * G * N * e : nullptr, D, dt_bias,
-                               dt_min, dt_max, h0 ? h0 + i * state : nullptr, yb ? yb + t0 * H * P * e : nullptr,
-                               h_final ? h_final + i * state : nullptr, 1, len, H, P, G, N, chunk, dtype, workspace,
-                               workspace_bytes, stream);
+        s = prefill(xb ? xb + t0 * H * P * e : nullptr, dtb ? dtb + t0 * H * e : nullptr, A_log,
+                    bb ? bb + t0 * G * N * e : nullptr, cb ? cb + t0 * G * N * e : nullptr, D, dt_bias, dt_min, dt_max,
+                    h0 ? h0 + i * state : nullptr, yb ? yb + t0 * H * P * e : nullptr,
+                    h_final ? h_final + i * state : nullptr, 1, len, H, P, G, N, chunk, dtype, workspace,
+                    workspace_bytes, stream, false);
         if (s != SSD_OK) return s;
     }
     return SSD_OK;
 }
 
 int ssd_chunk_scan_status(const void *workspace, void *stream) {
-    if (!workspace) return SSD_ERR_INVALID_ARG;
+    if (!workspace) {  // the built-in scratch of the allocation-free entry, on the current device
+        void *p = nullptr;
+        const cudaError_t e = ssd::noalloc_scratch(&p);
+        if (e != cudaSuccess) return cuda_status(e);
+        workspace = p;
+    }
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_status(e);
     int v = 0;

@@ -8,9 +8,9 @@
 // Autoregressive Caching for Inference" (bqwf.cn) §2.1: a fixed-size (kernel_size - 1)
 // input cache for the depthwise conv, kept beside the SSM state.
 //
-// One thread per (16-byte group of channels, 32-token strip): 8 bf16 or 4 fp32 channels, so
-// every load and store is a 16-byte vector and a warp moves 512 contiguous bytes per
-// instruction.  The thread keeps the K-1 previous inputs of its channels in registers and
+// One thread per (group of 4 channels, 32-token strip): 4 bf16 channels as one 8-byte vector,
+// or 4 fp32 channels as one 16-byte vector, so a warp moves 256 (bf16) or 512 (fp32)
+// contiguous bytes per instruction.  The thread keeps the K-1 previous inputs of its channels in registers and
 // slides along the strip, requesting 8 tokens' vectors at once before using any of them, so a
 // strip costs a few memory round trips rather than one per token.  Each input is read once,
 // plus K-1 halo tokens per strip (about 9 %, mostly from L2).  Launched with programmatic

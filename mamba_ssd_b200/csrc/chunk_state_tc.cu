@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_s, const __nv_bfloat16 *__restrict__ dt, const float *__restrict__ A_log,
     const float *__restrict__ dt_bias, float dt_min, float dt_max, float *__restrict__ dtf,
-    float *__restrict__ acs, int *__restrict__ status, int L, int H, int G, int nk, int total) {
+    float *__restrict__ acs, int *__restrict__ status, int reset_status, int L, int H, int G, int nk, int total) {
     using namespace cst;
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
@@ -127,8 +127,9 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     dtf = after_wait(dtf);
     acs = after_wait(acs);
     status = after_wait(status);
-    // this call's status word starts clean (a later wait of the call may record a timeout)
-    if (blockIdx.x == 0 && tid == 0) *status = SSD_OK;
+    // this call's status word starts clean (a later wait of the call may record a timeout),
+    // unless the caller keeps one word across several calls (the varlen prefill)
+    if (reset_status && blockIdx.x == 0 && tid == 0) *status = SSD_OK;
 
     auto stage = [&](int j) { return smem + kOffStage + (uint32_t)(j % kStages) * kStageBytes; };
     // a bounded wait that gives up at once when another role has already timed out
@@ -381,8 +382,8 @@ bool prefill_tc_supported(int dtype, int P, int N) {
 
 cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
                                   const float *dt_bias, float dt_min, float dt_max, float *dtf, float *acs,
-                                  float *states, int *status, int B, int L, int H, int G, int num_sms,
-                                  cudaStream_t st) {
+                                  float *states, int *status, bool reset_status, int B, int L, int H, int G,
+                                  int num_sms, cudaStream_t st) {
     using namespace cst;
     const int nk = cdiv(L, R);
     const int total = B * nk * H;
@@ -400,7 +401,7 @@ cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const void *dt,
     e = raise_smem_limit<chunk_state_tc_kernel>((int)kSmem);
     if (e != cudaSuccess) return e;
     return launch_pdl(chunk_state_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, tm_x, tm_b, tm_s,
-                      (const __nv_bfloat16 *)dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, status, L, H, G, nk,
+                      (const __nv_bfloat16 *)dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, status, reset_status ? 1 : 0, L, H, G, nk,
                       total);
 }
 

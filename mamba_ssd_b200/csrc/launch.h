@@ -69,7 +69,8 @@ size_t prefill_workspace_bytes(int B, int L, int H, int P, int N, int block, boo
 PrefillWorkspace carve_prefill_workspace(void *base, int B, int L, int H, int P, int N, int block,
                                          bool transposed_bf16);
 
-// Step a1 for the CUDA-core path: writes dt and acs (natural form) and resets the status word.
+// Step a1 for the CUDA-core path: writes dt and acs (natural form) and resets the status word
+// (when status is not NULL).
 cudaError_t launch_decay_prep(int dtype, const void *dt, const float *A_log, const float *dt_bias,
                               float dt_min, float dt_max, float *dtf, float *acs, int *status, int B,
                               int L, int H, int chunk, cudaStream_t st);
@@ -81,8 +82,8 @@ bool prefill_tc_supported(int dtype, int P, int N);
 // resets the status word: it is the first kernel of a tensor-core prefill call.
 cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
                                   const float *dt_bias, float dt_min, float dt_max, float *dtf, float *acs,
-                                  float *states, int *status, int B, int L, int H, int G, int num_sms,
-                                  cudaStream_t st);
+                                  float *states, int *status, bool reset_status, int B, int L, int H, int G,
+                                  int num_sms, cudaStream_t st);
 
 cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, const float *dtf,
                                  const float *acs, const __nv_bfloat16 *hT, const float *D, void *y,
@@ -111,7 +112,8 @@ size_t fused_workspace_bytes(int B, int L, int H);
 FusedWorkspace carve_fused_workspace(void *base, int B, int L, int H);
 cudaError_t launch_run_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
                                 const float *dt_bias, float dt_min, float dt_max, float *slots, float *decays,
-                                int *status, int B, int L, int H, int G, const RunLayout &lay, cudaStream_t st);
+                                int *status, bool reset_status, int B, int L, int H, int G, const RunLayout &lay,
+                                cudaStream_t st);
 cudaError_t launch_run_pass(float *slots, const float *decays, const float *h0, float *h_final, int B, int H,
                             const RunLayout &lay, cudaStream_t st);
 cudaError_t launch_chunk_scan_fused(const void *x, const void *Bm, const void *Cm, const void *dt, const float *A_log,
@@ -150,6 +152,10 @@ cudaError_t launch_gated_rmsnorm(int dtype, const void *y, const void *z, const 
 cudaError_t launch_causal_conv1d(int dtype, const void *xBC, const void *conv_w,
                                  const void *conv_b, void *out, void *conv_state_out, int B,
                                  int L, int Cc, int K, cudaStream_t st);
+
+// Device address, on the current device, of the built-in scratch array of
+// ssd_chunk_scan_fwd_noalloc (its first 256 bytes hold that entry's status word).
+cudaError_t noalloc_scratch(void **out);
 
 // One warp waits on an mbarrier that nothing arrives at, for limit_us microseconds, and records
 // SSD_ERR_TIMEOUT in *status (the bounded-wait self-test).

@@ -11,8 +11,6 @@
 //
 // The kernels, their launch order and their results are exactly those of
 // ssd_chunk_scan_fwd; only the scratch pointer differs.
-#include <mutex>
-
 #include "common.cuh"
 #include "launch.h"
 
@@ -25,28 +23,22 @@ static_assert(kScratchBytes % 256 == 0, "scratch size must keep 256-byte alignme
 // device array: its device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void *g_dev_ptr[kMaxDevices] = {};
+}  // namespace
 
-// Device address of the scratch array on the current device, looked up once per device.
-cudaError_t scratch_on_current_device(void **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+namespace ssd {
+// Device address of the scratch array on the current device, looked up on every call: it is
+// cheap once the library's module is loaded, and stays right across a device reset, which
+// reloads the module (possibly at another address).  With lazy module loading (the CUDA
+// default) the first lookup on a device loads the module, which is when the array's memory
+// is committed on that device.
+cudaError_t noalloc_scratch(void **out) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_dev_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_dev_ptr[dev] = p;
-    }
-    *out = g_dev_ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
-
-}  // namespace
+}  // namespace ssd
 
 extern "C" int ssd_chunk_scan_fwd_noalloc(const void *x, const void *dt, const float *A_log,
                                           const void *Bm, const void *Cm, const float *D,
@@ -61,7 +53,7 @@ extern "C" int ssd_chunk_scan_fwd_noalloc(const void *x, const void *dt, const f
         return ssd_chunk_scan_fwd(x, dt, A_log, Bm, Cm, D, dt_bias, dt_min, dt_max, h0, y, h_final, B,
                                   L, H, P, G, N, chunk, dtype, nullptr, 0, stream);
     void *scratch = nullptr;
-    const cudaError_t e = scratch_on_current_device(&scratch);
+    const cudaError_t e = ssd::noalloc_scratch(&scratch);
     if (e != cudaSuccess) return SSD_ERR_CUDA;
     // Nothing in the scratch has to start at zero: the prefill overwrites every byte it reads
     // (its status word is reset by the call's first kernel).

@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(rst::kThreads, 1) run_state_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_s, const __nv_bfloat16 *__restrict__ dt, const float *__restrict__ A_log,
     const float *__restrict__ dt_bias, float dt_min, float dt_max, float *__restrict__ decay_out,
-    int *__restrict__ status, int L, int H, int G, RunLayout lay) {
+    int *__restrict__ status, int reset_status, int L, int H, int G, RunLayout lay) {
     using namespace rst;
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
@@ -145,8 +145,9 @@ __global__ void __launch_bounds__(rst::kThreads, 1) run_state_tc_kernel(
     dt_bias = after_wait(dt_bias);
     decay_out = after_wait(decay_out);
     status = after_wait(status);
-    // the first kernel of the call: its status word starts clean
-    if (blockIdx.x == 0 && tid == 0) *status = SSD_OK;
+    // the first kernel of the call: its status word starts clean, unless the caller keeps one
+    // word across several calls (the varlen prefill)
+    if (reset_status && blockIdx.x == 0 && tid == 0) *status = SSD_OK;
 
     auto stage = [&](int j) { return smem + kOffStage + (uint32_t)(j % kStages) * kStageBytes; };
     auto wait = [&](uint64_t *bar, uint32_t parity) {
@@ -382,7 +383,8 @@ __global__ void __launch_bounds__(rst::kThreads, 1) run_state_tc_kernel(
 
 cudaError_t launch_run_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
                                 const float *dt_bias, float dt_min, float dt_max, float *slots, float *decays,
-                                int *status, int B, int L, int H, int G, const RunLayout &lay, cudaStream_t st) {
+                                int *status, bool reset_status, int B, int L, int H, int G, const RunLayout &lay,
+                                cudaStream_t st) {
     using namespace rst;
     CUtensorMap tm_x, tm_b, tm_s;
     cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B,
@@ -397,7 +399,8 @@ cudaError_t launch_run_state_tc(const void *x, const void *Bm, const void *dt, c
     e = raise_smem_limit<run_state_tc_kernel>((int)kSmem);
     if (e != cudaSuccess) return e;
     return launch_pdl(run_state_tc_kernel, dim3(lay.grid), dim3(kThreads), kSmem, st, tm_x, tm_b, tm_s,
-                      (const __nv_bfloat16 *)dt, A_log, dt_bias, dt_min, dt_max, decays, status, L, H, G, lay);
+                      (const __nv_bfloat16 *)dt, A_log, dt_bias, dt_min, dt_max, decays, status, reset_status ? 1 : 0, L, H, G,
+                      lay);
 }
 
 }  // namespace ssd

@@ -55,3 +55,16 @@ def test_varlen_rejects_misaligned_dt_rows():
     with pytest.raises(ssd.SSDError):
         ssd.ssd_chunk_scan_varlen_fwd(dev(inp["x"][0][0]), dev(inp["dt"][0][0]), dev(inp["A_log"][0]),
                                       dev(inp["Bm"][0][0]), dev(inp["Cm"][0][0]), cu)
+
+
+@pytest.mark.parametrize("lengths", [[300, 0], [0, 0], [129, 5]])
+def test_varlen_status_reset_once_per_call(lengths):
+    # the call resets the workspace status word itself (stale contents do not survive), also
+    # when its last sequence, or every sequence, is empty and launches no kernel that would
+    cu, inp, _ = _case(lengths, 8, 1, 128, "bf16", seed=11, with_h0=False)
+    T = int(cu[-1])
+    need = ssd.ssd_chunk_scan_workspace_size(1, max(lengths), 8, 64, 1, 128, 256, torch.bfloat16)
+    ws = torch.full((max(need, 256),), 0xFF, device="cuda", dtype=torch.uint8)
+    ssd.ssd_chunk_scan_varlen_fwd(dev(inp["x"][0][0]), dev(inp["dt"][0][0]), dev(inp["A_log"][0]),
+                                  dev(inp["Bm"][0][0]), dev(inp["Cm"][0][0]), cu, workspace=ws)
+    assert ssd.ssd_chunk_scan_status(ws) == 0, T
