@@ -735,6 +735,76 @@ def bench_block_conv(torch, ssd, device, peaks, launches=64, buffers=8):
             "frac": nbytes / per_launch_s / 1e9 / peaks["hbm_gbs"], "launches_timed": launches}
 
 
+def bench_block_conv_prefill(torch, ssd, device, peaks, launches=16, buffers=8):
+    """The conv before the scan and the prefill in one call (ssd_conv_chunk_scan_fwd) on the 2.7B
+    layer -- raw xBC [1, 4096, 5376], K = 4 -- against the same work as separate calls: the conv
+    kernel, torch copies splitting its output into contiguous x, B and C, then the prefill.
+    `launches` layers cycle over `buffers` input sets (≈ 0.9 GB each way, above L2), each variant
+    captured in one graph; per-layer times.  Algorithmic bytes of the one-call path: xBC and dt
+    read, y written, the conv cache and h_final written."""
+    B, L, H, P, G, N, K = PF["B"], PF["L"], PF["H"], PF["P"], PF["G"], PF["N"], DEC["K"]
+    Cc = H * P + 2 * G * N
+    bf = torch.bfloat16
+    g = torch.Generator(device=device)
+    g.manual_seed(PF["seed"] + 79)
+    scale = torch.ones(Cc, device=device)
+    scale[H * P:] = 1.0 / math.sqrt(N)
+    sets = [dict(xbc=(torch.randn((B, L, Cc), generator=g, device=device) * scale).to(bf),
+                 dt=(torch.randn((B, L, H), generator=g, device=device) - 2.0).to(bf),
+                 y=torch.empty((B, L, H, P), device=device, dtype=bf),
+                 hf=torch.empty((B, H, P, N), device=device, dtype=torch.float32),
+                 cs=torch.empty((B, Cc, K - 1), device=device, dtype=bf)) for _ in range(buffers)]
+    w = ((torch.rand((Cc, K), generator=g, device=device) * 2 - 1) / math.sqrt(K)).to(bf)
+    bias = ((torch.rand((Cc,), generator=g, device=device) * 2 - 1) / math.sqrt(K)).to(bf)
+    A_log = torch.log(torch.rand((H,), generator=g, device=device) * 15.0 + 1.0)
+    D = torch.randn((H,), generator=g, device=device)
+    ws1 = torch.empty(ssd.ssd_conv_chunk_scan_workspace_size(B, L, H, P, G, N, K, PF["chunk"], bf),
+                      device=device, dtype=torch.uint8)
+    ws2 = torch.empty(ssd.ssd_chunk_scan_workspace_size(B, L, H, P, G, N, PF["chunk"], bf), device=device,
+                      dtype=torch.uint8)
+    u = torch.empty((B, L, Cc), device=device, dtype=bf)
+    xs, Bs, Cs = (torch.empty((B, L, H, P), device=device, dtype=bf), torch.empty((B, L, G, N), device=device, dtype=bf),
+                  torch.empty((B, L, G, N), device=device, dtype=bf))
+    stream = torch.cuda.Stream(device=device)
+
+    def one_call():
+        for i in range(launches):
+            st = sets[i % buffers]
+            ssd.ssd_conv_chunk_scan_fwd(st["xbc"], w, bias, st["dt"], A_log, H, P, G, N, D=D, chunk=PF["chunk"],
+                                        dt_min=1e-3, dt_max=0.1, y=st["y"], h_final=st["hf"], conv_state_out=st["cs"],
+                                        workspace=ws1)
+
+    def separate():
+        for i in range(launches):
+            st = sets[i % buffers]
+            ssd.ssd_causal_conv1d_fwd(st["xbc"], w, bias, out=u, conv_state_out=st["cs"])
+            xs.copy_(u[..., :H * P].view(B, L, H, P))
+            Bs.copy_(u[..., H * P:H * P + G * N].view(B, L, G, N))
+            Cs.copy_(u[..., H * P + G * N:].view(B, L, G, N))
+            ssd.ssd_chunk_scan_fwd(xs, st["dt"], A_log, Bs, Cs, D=D, chunk=PF["chunk"], dt_min=1e-3, dt_max=0.1,
+                                   y=st["y"], h_final=st["hf"], workspace=ws2)
+
+    res = {}
+    for name, fn in (("one_call", one_call), ("separate", separate)):
+        with torch.cuda.stream(stream):
+            fn()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            fn()
+        res[name] = time_graph(torch, graph, stream, reps=5) / launches * 1e3  # us per layer
+        del graph
+    del sets
+    nbytes = B * L * Cc * 2 + B * L * H * 2 + B * L * H * P * 2 + B * Cc * (K - 1) * 2 + B * H * P * N * 4
+    return {"kernel": "ssd_conv_chunk_scan_fwd",
+            "workload": f"B={B}, L={L}, {Cc} channels, K={K}, H={H}, P={P}, N={N}, bf16, one layer per launch",
+            "one_call_us": res["one_call"], "separate_us": res["separate"],
+            "speedup": res["separate"] / res["one_call"], "algorithmic_bytes": nbytes,
+            "gbs": nbytes / (res["one_call"] * 1e-6) / 1e9,
+            "frac": nbytes / (res["one_call"] * 1e-6) / 1e9 / peaks["hbm_gbs"],
+            "separate_note": "conv kernel, three torch copies splitting its output into x, B, C, then the prefill"}
+
+
 def time_graph(torch, graph, stream, reps):
     """Median CUDA-event time of `reps` replays of a captured graph, after one warm-up."""
     graph.replay()
@@ -933,7 +1003,8 @@ def main():
         by_context = bench_context_sweep(torch, ssd, device, rank)
         torch.cuda.empty_cache()
     block_steps = {"causal_conv1d": bench_block_conv(torch, ssd, device, peaks),
-                   "gated_rmsnorm": bench_block_norm(torch, ssd, device, peaks)}
+                   "gated_rmsnorm": bench_block_norm(torch, ssd, device, peaks),
+                   "conv_prefill": bench_block_conv_prefill(torch, ssd, device, peaks)}
     torch.cuda.empty_cache()
 
     e2e = None

@@ -51,6 +51,10 @@
  * (B, H, P, G, N), the workspace holds the step's conv outputs instead of arrival counters
  * and needs no zero-fill; the kernel timer knows "decode_conv"; ssd_gated_rmsnorm_fwd and
  * ssd_chunk_scan_varlen_fwd added.
+ * Version 4: ssd_conv_chunk_scan_fwd / ssd_conv_chunk_scan_workspace_size (conv and prefill in
+ * one call), ssd_segment_decay and ssd_state_combine (context-parallel prefill) added;
+ * ssd_chunk_scan_fwd takes y = NULL (state only); ssd_chunk_scan_status(NULL) reads the
+ * allocation-free entry's scratch.
  */
 #ifndef MAMBA_SSD_H
 #define MAMBA_SSD_H
@@ -107,7 +111,8 @@ SSD_API size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, 
  *   dt_bias  [H]           float      NULL = 0
  *   dt_min, dt_max                    clip range of dt (0 and +inf disable it)
  *   h0       [B, H, P, N]  float      initial state, NULL = zeros
- *   y        [B, L, H, P]  dtype      output
+ *   y        [B, L, H, P]  dtype      output; NULL = only h_final is computed (the state the
+ *                                      sequence leaves: the output kernels are skipped)
  *   h_final  [B, H, P, N]  float      state after token L-1 (h0 when L == 0); NULL = not written
  *   chunk                              tokens per chunk; the last chunk may be ragged
  *   workspace, workspace_bytes         >= ssd_chunk_scan_workspace_size(...), 256-byte
@@ -127,6 +132,66 @@ SSD_API int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log
                        float dt_max, const float *h0, void *y, float *h_final, int B, int L,
                        int H, int P, int G, int N, int chunk, int dtype, void *workspace,
                        size_t workspace_bytes, void *stream);
+
+/*
+ * The block step before the scan and the chunked prefill in one call: raw conv inputs in, the
+ * scan's outputs and both caches out ([blog §2.1]: the depthwise sliding-window conv kept
+ * beside the state, its (kernel_size - 1) input cache; [blog §1.1, §1.2]: the chunked scan;
+ * [blog §3.2]: neighbouring element-wise work fused with the scan's data flow).
+ *   xBC            [B, L, Cc]    dtype  raw conv inputs, channels [x | B | C], Cc = H*P + 2*G*N
+ *   conv_w         [Cc, K]       dtype  depthwise taps, tap K-1 multiplies the newest input
+ *   conv_b         [Cc]          dtype  conv bias, NULL = 0
+ *   dt, A_log, D, dt_bias, dt_min, dt_max, h0, chunk, dtype   as for ssd_chunk_scan_fwd
+ *   y              [B, L, H, P]  dtype  output of the scan over x, B, C = SiLU(conv(xBC) + b)
+ *   h_final        [B, H, P, N]  float  NULL = not written
+ *   conv_state_out [B, Cc, K-1]  dtype  the last K-1 raw inputs, oldest first, zeros before the
+ *                                       start: with h_final, the cache ssd_decode_step continues
+ *                                       from; NULL = not written
+ *   workspace      >= ssd_conv_chunk_scan_workspace_size(...) bytes, 256-byte aligned
+ * The workspace holds the prefill's scratch (first, so ssd_chunk_scan_status(workspace, ...)
+ * reads this call's status) and then the conv output u [B, L, Cc]; the prefill kernels read
+ * x, B and C as strided views of u (token rows Cc elements apart) right after the conv kernel
+ * has written it, without splitting or copying it.  Supported: the shapes of
+ * ssd_chunk_scan_fwd and of ssd_causal_conv1d_fwd (2 <= K <= 8, Cc % 8 == 0, B <= 65535).
+ * Errors and ordering rules as for ssd_chunk_scan_fwd (everything checked before the first
+ * launch).
+ */
+SSD_API size_t ssd_conv_chunk_scan_workspace_size(int B, int L, int H, int P, int G, int N, int K, int chunk,
+                                                  int dtype);
+SSD_API int ssd_conv_chunk_scan_fwd(const void *xBC, const void *conv_w, const void *conv_b, const void *dt,
+                                    const float *A_log, const float *D, const float *dt_bias, float dt_min,
+                                    float dt_max, const float *h0, void *y, float *h_final, void *conv_state_out,
+                                    int B, int L, int H, int P, int G, int N, int K, int chunk, int dtype,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Context-parallel prefill: the sequence split into W consecutive segments, segment r on its
+ * own GPU ([blog §1.1]: chunks computed in parallel, the state passed between them by a light
+ * sequential scan; the segments are the chunks of that scan, one per GPU).  The recurrence is
+ * linear in the state, so segment r maps its incoming state h_in to
+ *   exp(sum_{t in segment} dt_t A) h_in + S_r,
+ * with S_r the state it leaves when started from zero (ssd_chunk_scan_fwd with y = NULL and
+ * h0 = NULL).  The steps per GPU: S_r and ssd_segment_decay; one all-gather of both over the
+ * GPUs (NCCL, outside this library); ssd_state_combine for the segment's carry-in; then
+ * ssd_chunk_scan_fwd over the segment from that carry-in (h0), which gives the segment's y.
+ * ssd_state_combine with r = W gives the state after the whole sequence on every GPU.
+ *
+ * ssd_segment_decay: log2 of each (batch, head) segment's total decay,
+ *   log2_decay[b, h] = -exp(A_log[h]) * sum_t clip(softplus(dt[b,t,h] + dt_bias[h]), dt_min, dt_max) * log2(e)
+ *   dt [B, L, H] dtype (raw); A_log, dt_bias [H] float (dt_bias nullable); log2_decay [B, H] float.
+ *   L = 0 gives 0.  Errors: SSD_ERR_INVALID_ARG for bad sizes, dtype, clip range or pointers.
+ *
+ * ssd_state_combine: the state entering segment r,
+ *   h = h0 (or 0);  for j = 0 .. r-1:  h = exp2(log2_decays[j]) * h + states[j];  out = h
+ *   states [r, B, H, P, N] float (the gathered S_j), log2_decays [r, B, H] float, h0 and out
+ *   [B, H, P, N] float (h0 nullable; out must not overlap the inputs).  r = 0 copies h0 (or
+ *   zeros).  Errors: SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED if P*N is not a multiple of 4.
+ * Both are asynchronous on `stream` like every other entry point.
+ */
+SSD_API int ssd_segment_decay(const void *dt, const float *A_log, const float *dt_bias, float dt_min, float dt_max,
+                              float *log2_decay, int B, int L, int H, int dtype, void *stream);
+SSD_API int ssd_state_combine(const float *states, const float *log2_decays, const float *h0, float *out, int r,
+                              int B, int H, int P, int N, void *stream);
 
 /*
  * Varlen prefill: n_seq sequences of different lengths packed into one token stream, each
@@ -309,8 +374,9 @@ SSD_API int ssd_selftest_wait_timeout(int *status, int limit_us, void *stream);
  * ssd_kernel_timer_enable(1) makes every later kernel launch on this process record a
  * pair of CUDA events around itself on its own stream; ssd_kernel_timer_read(name, ...)
  * waits for the recorded events of kernel `name` ("decay_prep", "chunk_state",
- * "state_pass", "chunk_scan", "decode_conv", "decode_step" (the decode state update),
- * "causal_conv1d", "gated_rmsnorm"), returns the summed
+ * "state_pass", "chunk_scan", "run_state", "run_pass", "chunk_scan_fused", "decode_conv",
+ * "decode_step" (the decode state update), "causal_conv1d", "gated_rmsnorm", "segment_decay",
+ * "state_combine"), returns the summed
  * device time in milliseconds and the number of launches timed, and forgets them.
  * Do not enable the timer while a stream is being captured into a CUDA graph.
  * Returns SSD_OK, SSD_ERR_INVALID_ARG for an unknown name, SSD_ERR_CUDA on an event error.

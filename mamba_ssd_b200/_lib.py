@@ -31,6 +31,11 @@ SIGNATURES = {
     "ssd_chunk_scan_fwd": (_i, [_vp, _vp, _fp, _vp, _vp, _fp, _fp, _f, _f, _fp, _vp, _fp]
                            + [_i] * 8 + [_vp, _sz, _vp]),
     "ssd_chunk_scan_status": (_i, [_vp, _vp]),
+    "ssd_conv_chunk_scan_workspace_size": (_sz, [_i] * 9),
+    "ssd_segment_decay": (_i, [_vp, _fp, _fp, _f, _f, _fp, _i, _i, _i, _i, _vp]),
+    "ssd_state_combine": (_i, [_fp, _fp, _fp, _fp, _i, _i, _i, _i, _i, _vp]),
+    "ssd_conv_chunk_scan_fwd": (_i, [_vp, _vp, _vp, _vp, _fp, _fp, _fp, _f, _f, _fp, _vp, _fp, _vp]
+                                + [_i] * 9 + [_vp, _sz, _vp]),
     "ssd_chunk_scan_varlen_fwd": (_i, [_vp, _vp, _fp, _vp, _vp, _fp, _fp, _f, _f, _fp, _vp, _fp, _vp]
                                   + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_chunk_scan_fwd_noalloc": (_i, [_vp, _vp, _fp, _vp, _vp, _fp, _fp, _f, _f, _fp, _vp, _fp]

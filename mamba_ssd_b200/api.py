@@ -54,8 +54,9 @@ def ssd_chunk_scan_workspace_size(B, L, H, P, G, N, chunk=256, dtype=torch.bfloa
 
 def ssd_chunk_scan_fwd(x, dt, A_log, Bm, Cm, D=None, chunk=256, h0=None, dt_bias=None,
                        dt_min=0.0, dt_max=math.inf, y=None, h_final=None, workspace=None,
-                       want_h_final=True, stream=None):
-    """Chunked SSD prefill.  Returns (y, h_final); h_final is None if not wanted."""
+                       want_h_final=True, want_y=True, stream=None):
+    """Chunked SSD prefill.  Returns (y, h_final); h_final is None if not wanted, y is None
+    when want_y is False (then only the state the sequence leaves is computed)."""
     Bsz, L, H, P = x.shape
     G, N = Bm.shape[2], Bm.shape[3]
     dt_code = _dtype_code(x)
@@ -67,7 +68,7 @@ def ssd_chunk_scan_fwd(x, dt, A_log, Bm, Cm, D=None, chunk=256, h0=None, dt_bias
     _need(D, "D", torch.float32, (H,))
     _need(dt_bias, "dt_bias", torch.float32, (H,))
     _need(h0, "h0", torch.float32, (Bsz, H, P, N))
-    if y is None:
+    if y is None and want_y:
         y = torch.empty_like(x)
     _need(y, "y", x.dtype, x.shape)
     if h_final is None and want_h_final:
@@ -83,6 +84,85 @@ def ssd_chunk_scan_fwd(x, dt, A_log, Bm, Cm, D=None, chunk=256, h0=None, dt_bias
         _stream(stream))
     check(s, "ssd_chunk_scan_fwd")
     return y, h_final
+
+
+def ssd_conv_chunk_scan_workspace_size(B, L, H, P, G, N, K, chunk=256, dtype=torch.bfloat16):
+    return int(_lib.lib().ssd_conv_chunk_scan_workspace_size(B, L, H, P, G, N, K, chunk, _DTYPES[dtype]))
+
+
+def ssd_conv_chunk_scan_fwd(xBC, conv_w, conv_b, dt, A_log, H, P, G, N, D=None, chunk=256, h0=None,
+                            dt_bias=None, dt_min=0.0, dt_max=math.inf, y=None, h_final=None,
+                            conv_state_out=None, want_h_final=True, want_state=True, workspace=None,
+                            stream=None):
+    """Causal conv + SiLU of the raw xBC [B, L, Cc] (channels [x | B | C]) and the chunked SSD
+    prefill over its output, in one call.  Returns (y [B,L,H,P], h_final [B,H,P,N] or None,
+    conv_state_out [B,Cc,K-1] or None)."""
+    Bsz, L, Cc = xBC.shape
+    K = conv_w.shape[1]
+    code = _dtype_code(xBC)
+    if Cc != H * P + 2 * G * N:
+        raise ValueError(f"xBC has {Cc} channels, expected H*P + 2*G*N = {H * P + 2 * G * N}")
+    _need(xBC, "xBC")
+    _need(conv_w, "conv_w", xBC.dtype, (Cc, K))
+    _need(conv_b, "conv_b", xBC.dtype, (Cc,))
+    _need(dt, "dt", xBC.dtype, (Bsz, L, H))
+    _need(A_log, "A_log", torch.float32, (H,))
+    _need(D, "D", torch.float32, (H,))
+    _need(dt_bias, "dt_bias", torch.float32, (H,))
+    _need(h0, "h0", torch.float32, (Bsz, H, P, N))
+    if y is None:
+        y = torch.empty((Bsz, L, H, P), device=xBC.device, dtype=xBC.dtype)
+    _need(y, "y", xBC.dtype, (Bsz, L, H, P))
+    if h_final is None and want_h_final:
+        h_final = torch.empty((Bsz, H, P, N), device=xBC.device, dtype=torch.float32)
+    _need(h_final, "h_final", torch.float32, (Bsz, H, P, N))
+    if conv_state_out is None and want_state:
+        conv_state_out = torch.empty((Bsz, Cc, K - 1), device=xBC.device, dtype=xBC.dtype)
+    _need(conv_state_out, "conv_state_out", xBC.dtype, (Bsz, Cc, K - 1))
+    need = _lib.lib().ssd_conv_chunk_scan_workspace_size(Bsz, L, H, P, G, N, K, chunk, code)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), device=xBC.device, dtype=torch.uint8)
+    s = _lib.lib().ssd_conv_chunk_scan_fwd(
+        _ptr(xBC), _ptr(conv_w), _ptr(conv_b), _ptr(dt), _ptr(A_log), _ptr(D), _ptr(dt_bias),
+        float(dt_min), float(dt_max), _ptr(h0), _ptr(y), _ptr(h_final), _ptr(conv_state_out),
+        Bsz, L, H, P, G, N, K, int(chunk), code, _ptr(workspace), workspace.numel(), _stream(stream))
+    check(s, "ssd_conv_chunk_scan_fwd")
+    return y, h_final, conv_state_out
+
+
+def ssd_segment_decay(dt, A_log, dt_bias=None, dt_min=0.0, dt_max=math.inf, out=None, stream=None):
+    """log2 of each (batch, head) segment's total decay, A_h * sum_t dt_t * log2(e), for dt
+    [B, L, H] (raw).  Returns out [B, H] float32."""
+    Bsz, L, H = dt.shape
+    code = _dtype_code(dt)
+    _need(dt, "dt")
+    _need(A_log, "A_log", torch.float32, (H,))
+    _need(dt_bias, "dt_bias", torch.float32, (H,))
+    if out is None:
+        out = torch.empty((Bsz, H), device=dt.device, dtype=torch.float32)
+    _need(out, "out", torch.float32, (Bsz, H))
+    check(_lib.lib().ssd_segment_decay(_ptr(dt), _ptr(A_log), _ptr(dt_bias), float(dt_min), float(dt_max),
+                                       _ptr(out), Bsz, L, H, code, _stream(stream)), "ssd_segment_decay")
+    return out
+
+
+def ssd_state_combine(states, log2_decays, r, h0=None, out=None, stream=None):
+    """The state entering segment r of a split sequence: h = h0 (or 0), then
+    h = exp2(log2_decays[j]) h + states[j] for j < r.  states [W, B, H, P, N] and log2_decays
+    [W, B, H] float32 hold every segment's own final state and decay; r = W gives the state
+    after the whole sequence.  Returns out [B, H, P, N]."""
+    W, Bsz, H, P, N = states.shape
+    if not 0 <= r <= W:
+        raise ValueError(f"r = {r} outside 0 .. {W}")
+    _need(states, "states", torch.float32)
+    _need(log2_decays, "log2_decays", torch.float32, (W, Bsz, H))
+    _need(h0, "h0", torch.float32, (Bsz, H, P, N))
+    if out is None:
+        out = torch.empty((Bsz, H, P, N), device=states.device, dtype=torch.float32)
+    _need(out, "out", torch.float32, (Bsz, H, P, N))
+    check(_lib.lib().ssd_state_combine(_ptr(states), _ptr(log2_decays), _ptr(h0), _ptr(out), int(r), Bsz, H, P,
+                                       N, _stream(stream)), "ssd_state_combine")
+    return out
 
 
 def ssd_chunk_scan_varlen_fwd(x, dt, A_log, Bm, Cm, cu_seqlens, D=None, chunk=256, h0=None,

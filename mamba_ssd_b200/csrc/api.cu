@@ -19,7 +19,8 @@ thread_local int g_last_cuda_error = 0;
 // ---- profiling hooks: launch counter and optional per-kernel CUDA-event timing ----
 const char *const kKernelNames[] = {"decay_prep",  "chunk_state",   "state_pass",  "chunk_scan",
                                     "decode_step", "causal_conv1d", "decode_conv", "gated_rmsnorm",
-                                    "run_state",   "run_pass",      "chunk_scan_fused"};
+                                    "run_state",   "run_pass",      "chunk_scan_fused", "segment_decay",
+                                    "state_combine"};
 enum KernelId {
     K_DECAY = 0,
     K_STATE,
@@ -32,6 +33,8 @@ enum KernelId {
     K_RSTATE,
     K_RPASS,
     K_FSCAN,
+    K_SEGDECAY,
+    K_COMBINE,
     K_COUNT
 };
 
@@ -239,7 +242,7 @@ const char *ssd_status_string(int status) {
 
 int ssd_last_cuda_error(void) { return g_last_cuda_error; }
 
-int ssd_abi_version(void) { return 3; }
+int ssd_abi_version(void) { return 4; }
 
 size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, int N, int chunk,
                                      int dtype) {
@@ -253,10 +256,13 @@ size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, int N, i
 namespace {
 // The prefill.  reset_status: the call's first kernel resets the workspace status word (a
 // single call); the varlen prefill resets it once itself and keeps it across its sequences.
+// x_row, bc_row: elements between consecutive tokens of x and of B / C (H*P and G*N when
+// dense; Cc when x, B and C are views into one conv output [.., Cc]).  y == NULL computes the
+// state only (h_final), skipping the output kernels.
 int prefill(const void *x, const void *dt, const float *A_log, const void *Bm, const void *Cm, const float *D,
             const float *dt_bias, float dt_min, float dt_max, const float *h0, void *y, float *h_final, int B, int L,
             int H, int P, int G, int N, int chunk, int dtype, void *workspace, size_t workspace_bytes, void *stream,
-            bool reset_status) {
+            bool reset_status, int64_t x_row, int64_t bc_row) {
     int s = check_prefill_shape(B, L, H, P, G, N, chunk, dtype);
     if (s != SSD_OK) return s;
     if ((s = check_dt_range(dt_min, dt_max)) != SSD_OK) return s;
@@ -265,10 +271,11 @@ int prefill(const void *x, const void *dt, const float *A_log, const void *Bm, c
         !opt_aligned16(h0) || !opt_aligned16(h_final))
         return SSD_ERR_INVALID_ARG;
     if (L > 0) {
-        if (!x || !dt || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
-        if (!aligned16(x) || !aligned16(dt) || !aligned16(Bm) || !aligned16(Cm) || !aligned16(y))
+        if (!x || !dt || !Bm || (y && !Cm)) return SSD_ERR_INVALID_ARG;
+        if (!aligned16(x) || !aligned16(dt) || !aligned16(Bm) || !opt_aligned16(Cm) || !opt_aligned16(y))
             return SSD_ERR_INVALID_ARG;
     }
+    const bool want_y = y != nullptr;
     const size_t need = prefill_query_bytes(B, L, H, P, G, N, chunk, dtype);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return SSD_ERR_WORKSPACE;
@@ -280,15 +287,15 @@ int prefill(const void *x, const void *dt, const float *A_log, const void *Bm, c
         ssd::FusedWorkspace ws = ssd::carve_fused_workspace(workspace, B, L, H);
         e = timed_launch(K_RSTATE, st, [&] {
             return ssd::launch_run_state_tc(x, Bm, dt, A_log, dt_bias, dt_min, dt_max, ws.slots, ws.decays,
-                                            ws.status, reset_status, B, L, H, G, lay, st);
+                                            ws.status, reset_status, B, L, H, G, x_row, bc_row, lay, st);
         });
         if (e != cudaSuccess) return cuda_status(e);
         e = timed_launch(K_RPASS, st,
                          [&] { return ssd::launch_run_pass(ws.slots, ws.decays, h0, h_final, B, H, lay, st); });
-        if (e != cudaSuccess) return cuda_status(e);
+        if (e != cudaSuccess || !want_y) return cuda_status(e);
         e = timed_launch(K_FSCAN, st, [&] {
             return ssd::launch_chunk_scan_fused(x, Bm, Cm, dt, A_log, dt_bias, dt_min, dt_max, D, ws.slots, y,
-                                                ws.status, B, L, H, G, lay, st);
+                                                ws.status, B, L, H, G, x_row, bc_row, lay, st);
         });
         return cuda_status(e);
     }
@@ -300,7 +307,8 @@ int prefill(const void *x, const void *dt, const float *A_log, const void *Bm, c
             // the state kernel also forms the decay factors (step a1) of the items it owns
             e = timed_launch(K_STATE, st, [&] {
                 return ssd::launch_chunk_state_tc(x, Bm, dt, A_log, dt_bias, dt_min, dt_max, ws.dtf, ws.acs,
-                                                  ws.states, ws.status, reset_status, B, L, H, G, sm_count(), st);
+                                                  ws.states, ws.status, reset_status, B, L, H, G, x_row, bc_row,
+                                                  sm_count(), st);
             });
             if (e != cudaSuccess) return cuda_status(e);
         }
@@ -308,10 +316,10 @@ int prefill(const void *x, const void *dt, const float *A_log, const void *Bm, c
             return ssd::launch_state_pass_t(ws.states, ws.acs, h0, h_final, ws.hT, B, L, H, P, N, blk, st);
         });
         if (e != cudaSuccess) return cuda_status(e);
-        if (L > 0) {
+        if (L > 0 && want_y) {
             e = timed_launch(K_SCAN, st, [&] {
-                return ssd::launch_chunk_scan_tc(x, Bm, Cm, ws.dtf, ws.acs, ws.hT, D, y, ws.status, B, L, H, G,
-                                                 sm_count(), st);
+                return ssd::launch_chunk_scan_tc(x, Bm, Cm, ws.dtf, ws.acs, ws.hT, D, y, ws.status, B, L, H, G, x_row,
+                                                 bc_row, sm_count(), st);
             });
             if (e != cudaSuccess) return cuda_status(e);
         }
@@ -326,7 +334,8 @@ int prefill(const void *x, const void *dt, const float *A_log, const void *Bm, c
         });
         if (e != cudaSuccess) return cuda_status(e);
         e = timed_launch(K_STATE, st, [&] {
-            return ssd::launch_chunk_state(dtype, x, Bm, ws.dtf, ws.acs, ws.states, B, L, H, G, N, chunk, st);
+            return ssd::launch_chunk_state(dtype, x, Bm, ws.dtf, ws.acs, ws.states, B, L, H, G, N, chunk, x_row,
+                                           bc_row, st);
         });
         if (e != cudaSuccess) return cuda_status(e);
     }
@@ -334,10 +343,10 @@ int prefill(const void *x, const void *dt, const float *A_log, const void *Bm, c
         return ssd::launch_state_pass(ws.states, ws.acs, h0, h_final, B, L, H, P, N, chunk, st);
     });
     if (e != cudaSuccess) return cuda_status(e);
-    if (L > 0) {
+    if (L > 0 && want_y) {
         e = timed_launch(K_SCAN, st, [&] {
             return ssd::launch_chunk_scan(dtype, x, Bm, Cm, ws.dtf, ws.acs, ws.states, D, y, B, L, H, G, N,
-                                          chunk, st);
+                                          chunk, x_row, bc_row, st);
         });
         if (e != cudaSuccess) return cuda_status(e);
     }
@@ -353,7 +362,94 @@ int ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A_log, const 
                        float *h_final, int B, int L, int H, int P, int G, int N, int chunk, int dtype,
                        void *workspace, size_t workspace_bytes, void *stream) {
     return prefill(x, dt, A_log, Bm, Cm, D, dt_bias, dt_min, dt_max, h0, y, h_final, B, L, H, P, G, N, chunk,
-                   dtype, workspace, workspace_bytes, stream, true);
+                   dtype, workspace, workspace_bytes, stream, true, (int64_t)H * P, (int64_t)G * N);
+}
+
+// The prefill workspace first (so its status word is the workspace's first word), then the
+// conv output u [B, L, Cc].
+namespace {
+size_t conv_out_bytes(int B, int L, int Cc, int dtype) {
+    return ssd::align_up((size_t)B * L * Cc * (dtype == SSD_DTYPE_BF16 ? 2 : 4), 256);
+}
+int check_conv_shape(int B, int L, int Cc, int K) {
+    if (K < 2 || K > 8 || Cc % 8 != 0) return SSD_ERR_UNSUPPORTED;
+    if (B > 65535 || L > 65535 * 32) return SSD_ERR_UNSUPPORTED;  // grid z; 32-token strips on grid y
+    return SSD_OK;
+}
+}  // namespace
+
+size_t ssd_conv_chunk_scan_workspace_size(int B, int L, int H, int P, int G, int N, int K, int chunk, int dtype) {
+    if (check_prefill_shape(B, L, H, P, G, N, chunk, dtype) != SSD_OK || K <= 0) return 0;
+    const int Cc = H * P + 2 * G * N;
+    if (check_conv_shape(B, L, Cc, K) != SSD_OK || B == 0) return 0;
+    return prefill_query_bytes(B, L, H, P, G, N, chunk, dtype) + conv_out_bytes(B, L, Cc, dtype);
+}
+
+int ssd_conv_chunk_scan_fwd(const void *xBC, const void *conv_w, const void *conv_b, const void *dt,
+                            const float *A_log, const float *D, const float *dt_bias, float dt_min, float dt_max,
+                            const float *h0, void *y, float *h_final, void *conv_state_out, int B, int L, int H,
+                            int P, int G, int N, int K, int chunk, int dtype, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+    int s = check_prefill_shape(B, L, H, P, G, N, chunk, dtype);
+    if (s != SSD_OK) return s;
+    if (K <= 0) return SSD_ERR_INVALID_ARG;
+    const int Cc = H * P + 2 * G * N;
+    if ((s = check_conv_shape(B, L, Cc, K)) != SSD_OK) return s;
+    if ((s = check_dt_range(dt_min, dt_max)) != SSD_OK) return s;
+    if (B == 0) return SSD_OK;
+    if (!conv_w || !aligned16(conv_w) || !opt_aligned16(conv_b) || !opt_aligned16(conv_state_out) || !A_log ||
+        !aligned16(A_log) || !opt_aligned16(D) || !opt_aligned16(dt_bias) || !opt_aligned16(h0) ||
+        !opt_aligned16(h_final))
+        return SSD_ERR_INVALID_ARG;
+    if (L > 0 && (!xBC || !dt || !y || !aligned16(xBC) || !aligned16(dt) || !aligned16(y))) return SSD_ERR_INVALID_ARG;
+    const size_t pre_bytes = prefill_query_bytes(B, L, H, P, G, N, chunk, dtype);
+    const size_t need = pre_bytes + conv_out_bytes(B, L, Cc, dtype);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return SSD_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t e = dtype == SSD_DTYPE_BF16 ? 2 : 4;
+    char *u = static_cast<char *>(workspace) + pre_bytes;
+    cudaError_t ce = cudaSuccess;
+    if (L > 0) {
+        ce = timed_launch(K_CONV, st, [&] {
+            return ssd::launch_causal_conv1d(dtype, xBC, conv_w, conv_b, u, conv_state_out, B, L, Cc, K, st);
+        });
+    } else if (conv_state_out) {  // empty prefix: the cache is all zeros
+        ce = cudaMemsetAsync(conv_state_out, 0, (size_t)B * Cc * (K - 1) * e, st);
+    }
+    if (ce != cudaSuccess) return cuda_status(ce);
+    // x, B and C are strided views of u (token rows Cc elements apart): no split, no copy
+    return prefill(u, dt, A_log, u + (size_t)H * P * e, u + ((size_t)H * P + (size_t)G * N) * e, D, dt_bias, dt_min,
+                   dt_max, h0, y, h_final, B, L, H, P, G, N, chunk, dtype, workspace, pre_bytes, stream, true, Cc, Cc);
+}
+
+int ssd_segment_decay(const void *dt, const float *A_log, const float *dt_bias, float dt_min, float dt_max,
+                      float *log2_decay, int B, int L, int H, int dtype, void *stream) {
+    if (B < 0 || L < 0 || H <= 0) return SSD_ERR_INVALID_ARG;
+    if (dtype != SSD_DTYPE_F32 && dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
+    int s = check_dt_range(dt_min, dt_max);
+    if (s != SSD_OK) return s;
+    if (B == 0) return SSD_OK;
+    if (!A_log || !log2_decay || !aligned16(A_log) || !aligned16(log2_decay) || !opt_aligned16(dt_bias))
+        return SSD_ERR_INVALID_ARG;
+    if (L > 0 && (!dt || !aligned16(dt))) return SSD_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return cuda_status(timed_launch(K_SEGDECAY, st, [&] {
+        return ssd::launch_segment_decay(dtype, dt, A_log, dt_bias, dt_min, dt_max, log2_decay, B, L, H, st);
+    }));
+}
+
+int ssd_state_combine(const float *states, const float *log2_decays, const float *h0, float *out, int r, int B, int H,
+                      int P, int N, void *stream) {
+    if (r < 0 || B < 0 || H <= 0 || P <= 0 || N <= 0) return SSD_ERR_INVALID_ARG;
+    if (((size_t)P * N) % 4 != 0) return SSD_ERR_UNSUPPORTED;
+    if (B == 0) return SSD_OK;
+    if (!out || !aligned16(out) || !opt_aligned16(h0)) return SSD_ERR_INVALID_ARG;
+    if (r > 0 && (!states || !log2_decays || !aligned16(states) || !aligned16(log2_decays))) return SSD_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return cuda_status(timed_launch(K_COMBINE, st, [&] {
+        return ssd::launch_state_combine(states, log2_decays, h0, out, r, B, H, P, N, st);
+    }));
 }
 
 int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float *A_log, const void *Bm,
@@ -407,7 +503,7 @@ int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float *A_log,
                     bb ? bb + t0 * G * N * e : nullptr, cb ? cb + t0 * G * N * e : nullptr, D, dt_bias, dt_min, dt_max,
                     h0 ? h0 + i * state : nullptr, yb ? yb + t0 * H * P * e : nullptr,
                     h_final ? h_final + i * state : nullptr, 1, len, H, P, G, N, chunk, dtype, workspace,
-                    workspace_bytes, stream, false);
+                    workspace_bytes, stream, false, (int64_t)H * P, (int64_t)G * N);
         if (s != SSD_OK) return s;
     }
     return SSD_OK;

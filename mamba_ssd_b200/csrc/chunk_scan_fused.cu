@@ -603,17 +603,17 @@ bool prefill_fused_supported(int dtype, int P, int N, int H, int G) {
 cudaError_t launch_chunk_scan_fused(const void *x, const void *Bm, const void *Cm, const void *dt, const float *A_log,
                                     const float *dt_bias, float dt_min, float dt_max, const float *D,
                                     const float *slots, void *y, int *status, int B, int L, int H, int G,
-                                    const RunLayout &lay, cudaStream_t st) {
+                                    int64_t x_row, int64_t bc_row, const RunLayout &lay, cudaStream_t st) {
     using namespace csf;
     CUtensorMap tm_x, tm_b, tm_c, tm_y;
-    cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B,
-                                      (uint64_t)H * P * 2, (uint64_t)L * H * P * 2, 64, R, 1);
+    cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B, (uint64_t)x_row * 2,
+                                      (uint64_t)L * x_row * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16_3d(&tm_b, Bm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)G * N * 2,
-                          (uint64_t)L * G * N * 2, 64, R, 1);
+    e = make_tmap_bf16_3d(&tm_b, Bm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)bc_row * 2,
+                          (uint64_t)L * bc_row * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16_3d(&tm_c, Cm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)G * N * 2,
-                          (uint64_t)L * G * N * 2, 64, R, 1);
+    e = make_tmap_bf16_3d(&tm_c, Cm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)bc_row * 2,
+                          (uint64_t)L * bc_row * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
     e = make_tmap_bf16_3d(&tm_y, y, (uint64_t)H * P, (uint64_t)L, (uint64_t)B, (uint64_t)H * P * 2,
                           (uint64_t)L * H * P * 2, 64, R, 1);

@@ -379,19 +379,21 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
 
 cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, const float *dtf,
                                  const float *acs, const __nv_bfloat16 *hT, const float *D, void *y,
-                                 int *status, int B, int L, int H, int G, int num_sms, cudaStream_t st) {
+                                 int *status, int B, int L, int H, int G, int64_t x_row, int64_t bc_row, int num_sms,
+                                 cudaStream_t st) {
     using namespace csc;
     const int nk = cdiv(L, R);
     const int total = B * nk * H;
     CUtensorMap tm_x, tm_b, tm_c, tm_h, tm_y;
-    cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B,
-                                      (uint64_t)H * P * 2, (uint64_t)L * H * P * 2, 64, R, 1);
+    // x, B and C rows are x_row and bc_row elements apart (H*P and G*N when dense); y is dense
+    cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B, (uint64_t)x_row * 2,
+                                      (uint64_t)L * x_row * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16_3d(&tm_b, Bm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)G * N * 2,
-                          (uint64_t)L * G * N * 2, 64, R, 1);
+    e = make_tmap_bf16_3d(&tm_b, Bm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)bc_row * 2,
+                          (uint64_t)L * bc_row * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16_3d(&tm_c, Cm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)G * N * 2,
-                          (uint64_t)L * G * N * 2, 64, R, 1);
+    e = make_tmap_bf16_3d(&tm_c, Cm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)bc_row * 2,
+                          (uint64_t)L * bc_row * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
     e = make_tmap_bf16_2d(&tm_h, hT, (uint64_t)P, (uint64_t)B * nk * H * N, (uint64_t)P * 2, 64, R);
     if (e != cudaSuccess) return e;

@@ -32,7 +32,7 @@ template <typename T, int N>
 __global__ void __launch_bounds__(256) chunk_state_simt_kernel(
     const T *__restrict__ x, const T *__restrict__ Bm, const float *__restrict__ dtf,
     const float *__restrict__ acs, float *__restrict__ states, int L, int H, int G, int Q,
-    int nc) {
+    int nc, int64_t x_row, int64_t bc_row) {
     constexpr int NPT = N / 16;
     constexpr int SB = 32;  // tokens per stage
     __shared__ __align__(16) float Xs[SB][kP];
@@ -58,14 +58,14 @@ __global__ void __launch_bounds__(256) chunk_state_simt_kernel(
             float v = 0.f;
             if (tok < L) {
                 const float w = dt_row[s0 + s] * expf(a_last - acs_row[s0 + s]);
-                v = w * to_f(x[(((size_t)b * L + tok) * H + h) * kP + p]);
+                v = w * to_f(x[((size_t)b * L + tok) * x_row + (size_t)h * kP + p]);
             }
             Xs[s][p] = v;
         }
         for (int idx = tid; idx < SB * N; idx += 256) {
             const int s = idx / N, n = idx % N;
             const int tok = c * Q + s0 + s;
-            Bs[s][n] = tok < L ? to_f(Bm[(((size_t)b * L + tok) * G + g) * N + n]) : 0.f;
+            Bs[s][n] = tok < L ? to_f(Bm[((size_t)b * L + tok) * bc_row + (size_t)g * N + n]) : 0.f;
         }
         __syncthreads();
 #pragma unroll 4
@@ -106,7 +106,8 @@ template <typename T, int N>
 __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
     const T *__restrict__ x, const T *__restrict__ Bm, const T *__restrict__ Cm,
     const float *__restrict__ dtf, const float *__restrict__ acs, const float *__restrict__ hprev,
-    const float *__restrict__ D, T *__restrict__ y, int L, int H, int G, int Q, int nc) {
+    const float *__restrict__ D, T *__restrict__ y, int L, int H, int G, int Q, int nc, int64_t x_row,
+    int64_t bc_row) {
     extern __shared__ __align__(16) float smem[];
     float *Cs = smem;                  // [N][kLd]   C rows of the row block, transposed
     float *Bs = Cs + N * kLd;          // [N][kLd]   B rows of a column block, transposed
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
     for (int idx = tid; idx < 64 * N; idx += 256) {
         const int l = idx / N, n = idx % N;
         const int tok = c * Q + l0 + l;
-        Cs[n * kLd + l] = tok < L ? to_f(Cm[(((size_t)b * L + tok) * G + g) * N + n]) : 0.f;
+        Cs[n * kLd + l] = tok < L ? to_f(Cm[((size_t)b * L + tok) * bc_row + (size_t)g * N + n]) : 0.f;
     }
     if (tid < 64) acs_l[tid] = acs_row[l0 + tid];
 
@@ -145,13 +146,13 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
         for (int idx = tid; idx < 64 * N; idx += 256) {
             const int s = idx / N, n = idx % N;
             const int tok = c * Q + s0 + s;
-            Bs[n * kLd + s] = tok < L ? to_f(Bm[(((size_t)b * L + tok) * G + g) * N + n]) : 0.f;
+            Bs[n * kLd + s] = tok < L ? to_f(Bm[((size_t)b * L + tok) * bc_row + (size_t)g * N + n]) : 0.f;
         }
         for (int idx = tid; idx < 64 * kP; idx += 256) {
             const int s = idx / kP, p = idx % kP;
             const int tok = c * Q + s0 + s;
             Xs[s * kLd + p] =
-                tok < L ? dt_row[s0 + s] * to_f(x[(((size_t)b * L + tok) * H + h) * kP + p]) : 0.f;
+                tok < L ? dt_row[s0 + s] * to_f(x[((size_t)b * L + tok) * x_row + (size_t)h * kP + p]) : 0.f;
         }
         if (tid < 64) acs_s[tid] = acs_row[s0 + tid];
         __syncthreads();
@@ -229,11 +230,12 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
         const int tok = c * Q + l0 + l;
         if (tok >= L) continue;
         const float e = expf(acs_l[l]);
-        const size_t rowoff = (((size_t)b * L + tok) * H + h) * kP;
+        const size_t rowoff = (((size_t)b * L + tok) * H + h) * kP;  // y is dense
+        const size_t xoff = ((size_t)b * L + tok) * x_row + (size_t)h * kP;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int p = tx * 4 + j;
-            const float xv = to_f(x[rowoff + p]);
+            const float xv = to_f(x[xoff + p]);
             y[rowoff + p] = from_f<T>(acc[i][j] + e * off[i][j] + d * xv);
         }
     }
@@ -241,19 +243,20 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
 
 template <typename T, int N>
 static cudaError_t chunk_state_n(const void *x, const void *Bm, const float *dtf, const float *acs,
-                                 float *states, int B, int L, int H, int G, int chunk,
-                                 cudaStream_t st) {
+                                 float *states, int B, int L, int H, int G, int chunk, int64_t x_row,
+                                 int64_t bc_row, cudaStream_t st) {
     const int nc = cdiv(L, chunk);
     dim3 grid(nc, H, B);
     chunk_state_simt_kernel<T, N><<<grid, 256, 0, st>>>((const T *)x, (const T *)Bm, dtf, acs,
-                                                        states, L, H, G, chunk, nc);
+                                                        states, L, H, G, chunk, nc, x_row, bc_row);
     return cudaGetLastError();
 }
 
 template <typename T, int N>
 static cudaError_t chunk_scan_n(const void *x, const void *Bm, const void *Cm, const float *dtf,
                                 const float *acs, const float *hprev, const float *D, void *y,
-                                int B, int L, int H, int G, int chunk, cudaStream_t st) {
+                                int B, int L, int H, int G, int chunk, int64_t x_row, int64_t bc_row,
+                                cudaStream_t st) {
     const int nc = cdiv(L, chunk);
     dim3 grid(nc * (chunk / 64), H, B);
     constexpr size_t smem = chunk_scan_simt_smem<N>();
@@ -261,7 +264,7 @@ static cudaError_t chunk_scan_n(const void *x, const void *Bm, const void *Cm, c
     if (e != cudaSuccess) return e;
     chunk_scan_simt_kernel<T, N><<<grid, 256, smem, st>>>((const T *)x, (const T *)Bm,
                                                           (const T *)Cm, dtf, acs, hprev, D,
-                                                          (T *)y, L, H, G, chunk, nc);
+                                                          (T *)y, L, H, G, chunk, nc, x_row, bc_row);
     return cudaGetLastError();
 }
 
@@ -276,22 +279,24 @@ static cudaError_t chunk_scan_n(const void *x, const void *Bm, const void *Cm, c
 
 cudaError_t launch_chunk_state(int dtype, const void *x, const void *Bm, const float *dtf,
                                const float *acs, float *states, int B, int L, int H, int G, int N,
-                               int chunk, cudaStream_t st) {
+                               int chunk, int64_t x_row, int64_t bc_row, cudaStream_t st) {
     if (dtype == SSD_DTYPE_BF16) {
-        SSD_DISPATCH_N(N, chunk_state_n, __nv_bfloat16, x, Bm, dtf, acs, states, B, L, H, G, chunk, st)
+        SSD_DISPATCH_N(N, chunk_state_n, __nv_bfloat16, x, Bm, dtf, acs, states, B, L, H, G, chunk, x_row, bc_row,
+                       st)
     }
-    SSD_DISPATCH_N(N, chunk_state_n, float, x, Bm, dtf, acs, states, B, L, H, G, chunk, st)
+    SSD_DISPATCH_N(N, chunk_state_n, float, x, Bm, dtf, acs, states, B, L, H, G, chunk, x_row, bc_row, st)
 }
 
 cudaError_t launch_chunk_scan(int dtype, const void *x, const void *Bm, const void *Cm,
                               const float *dtf, const float *acs, const float *hprev,
                               const float *D, void *y, int B, int L, int H, int G, int N,
-                              int chunk, cudaStream_t st) {
+                              int chunk, int64_t x_row, int64_t bc_row, cudaStream_t st) {
     if (dtype == SSD_DTYPE_BF16) {
         SSD_DISPATCH_N(N, chunk_scan_n, __nv_bfloat16, x, Bm, Cm, dtf, acs, hprev, D, y, B, L, H,
-                       G, chunk, st)
+                       G, chunk, x_row, bc_row, st)
     }
-    SSD_DISPATCH_N(N, chunk_scan_n, float, x, Bm, Cm, dtf, acs, hprev, D, y, B, L, H, G, chunk, st)
+    SSD_DISPATCH_N(N, chunk_scan_n, float, x, Bm, Cm, dtf, acs, hprev, D, y, B, L, H, G, chunk, x_row, bc_row,
+                   st)
 }
 
 }  // namespace ssd

@@ -383,16 +383,17 @@ bool prefill_tc_supported(int dtype, int P, int N) {
 cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
                                   const float *dt_bias, float dt_min, float dt_max, float *dtf, float *acs,
                                   float *states, int *status, bool reset_status, int B, int L, int H, int G,
-                                  int num_sms, cudaStream_t st) {
+                                  int64_t x_row, int64_t bc_row, int num_sms, cudaStream_t st) {
     using namespace cst;
     const int nk = cdiv(L, R);
     const int total = B * nk * H;
     CUtensorMap tm_x, tm_b, tm_s;
-    cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B,
-                                      (uint64_t)H * P * 2, (uint64_t)L * H * P * 2, 64, R, 1);
+    // x and B rows are x_row and bc_row elements apart (H*P and G*N when dense)
+    cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B, (uint64_t)x_row * 2,
+                                      (uint64_t)L * x_row * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16_3d(&tm_b, Bm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)G * N * 2,
-                          (uint64_t)L * G * N * 2, 64, R, 1);
+    e = make_tmap_bf16_3d(&tm_b, Bm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)bc_row * 2,
+                          (uint64_t)L * bc_row * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
     // S^T of every item as rows of 64 fp32: TMA boxes of 32 columns x 128 rows
     e = make_tmap_f32_2d(&tm_s, states, (uint64_t)P, (uint64_t)total * N, (uint64_t)P * 4, 32, R);

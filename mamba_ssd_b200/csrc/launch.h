@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
+#include <stdint.h>
 
 #include <atomic>
 
@@ -83,11 +84,12 @@ bool prefill_tc_supported(int dtype, int P, int N);
 cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
                                   const float *dt_bias, float dt_min, float dt_max, float *dtf, float *acs,
                                   float *states, int *status, bool reset_status, int B, int L, int H, int G,
-                                  int num_sms, cudaStream_t st);
+                                  int64_t x_row, int64_t bc_row, int num_sms, cudaStream_t st);
 
 cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, const float *dtf,
                                  const float *acs, const __nv_bfloat16 *hT, const float *D, void *y,
-                                 int *status, int B, int L, int H, int G, int num_sms, cudaStream_t st);
+                                 int *status, int B, int L, int H, int G, int64_t x_row, int64_t bc_row, int num_sms,
+                                 cudaStream_t st);
 cudaError_t launch_state_pass_t(const float *states, const float *acs, const float *h0, float *h_final,
                                 __nv_bfloat16 *hT, int B, int L, int H, int P, int N, int chunk,
                                 cudaStream_t st);
@@ -112,18 +114,20 @@ size_t fused_workspace_bytes(int B, int L, int H);
 FusedWorkspace carve_fused_workspace(void *base, int B, int L, int H);
 cudaError_t launch_run_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
                                 const float *dt_bias, float dt_min, float dt_max, float *slots, float *decays,
-                                int *status, bool reset_status, int B, int L, int H, int G, const RunLayout &lay,
-                                cudaStream_t st);
+                                int *status, bool reset_status, int B, int L, int H, int G, int64_t x_row,
+                                int64_t bc_row, const RunLayout &lay, cudaStream_t st);
 cudaError_t launch_run_pass(float *slots, const float *decays, const float *h0, float *h_final, int B, int H,
                             const RunLayout &lay, cudaStream_t st);
 cudaError_t launch_chunk_scan_fused(const void *x, const void *Bm, const void *Cm, const void *dt, const float *A_log,
                                     const float *dt_bias, float dt_min, float dt_max, const float *D,
                                     const float *slots, void *y, int *status, int B, int L, int H, int G,
-                                    const RunLayout &lay, cudaStream_t st);
+                                    int64_t x_row, int64_t bc_row, const RunLayout &lay, cudaStream_t st);
 
+// x rows (tokens) are x_row elements apart and B/C rows bc_row apart: H*P and G*N when dense,
+// wider when x, B and C are strided views into one [.., H*P + 2*G*N] conv output.
 cudaError_t launch_chunk_state(int dtype, const void *x, const void *Bm, const float *dtf,
                                const float *acs, float *states, int B, int L, int H, int G, int N,
-                               int chunk, cudaStream_t st);
+                               int chunk, int64_t x_row, int64_t bc_row, cudaStream_t st);
 
 cudaError_t launch_state_pass(float *states, const float *acs, const float *h0, float *h_final,
                               int B, int L, int H, int P, int N, int chunk, cudaStream_t st);
@@ -131,7 +135,7 @@ cudaError_t launch_state_pass(float *states, const float *acs, const float *h0, 
 cudaError_t launch_chunk_scan(int dtype, const void *x, const void *Bm, const void *Cm,
                               const float *dtf, const float *acs, const float *hprev,
                               const float *D, void *y, int B, int L, int H, int G, int N,
-                              int chunk, cudaStream_t st);
+                              int chunk, int64_t x_row, int64_t bc_row, cudaStream_t st);
 
 // One decode step is two launches: the conv kernel (conv, SiLU, conv-cache roll, dt and the
 // decay factor, into u_ws [B][Cc] fp32 and da_ws [B][H] (dt, a)), then the state kernel.
@@ -152,6 +156,13 @@ cudaError_t launch_gated_rmsnorm(int dtype, const void *y, const void *z, const 
 cudaError_t launch_causal_conv1d(int dtype, const void *xBC, const void *conv_w,
                                  const void *conv_b, void *out, void *conv_state_out, int B,
                                  int L, int Cc, int K, cudaStream_t st);
+
+// Context-parallel steps: each (batch, head) segment's total decay, log2 form, into out [B][H];
+// and the carry-in h = h0 (or 0), h = exp2(ld_j) h + S_j for j < r, of [B][H][P][N] states.
+cudaError_t launch_segment_decay(int dtype, const void *dt, const float *A_log, const float *dt_bias, float dt_min,
+                                 float dt_max, float *out, int B, int L, int H, cudaStream_t st);
+cudaError_t launch_state_combine(const float *states, const float *log2_decays, const float *h0, float *out, int r,
+                                 int B, int H, int P, int N, cudaStream_t st);
 
 // Device address, on the current device, of the built-in scratch array of
 // ssd_chunk_scan_fwd_noalloc (its first 256 bytes hold that entry's status word).

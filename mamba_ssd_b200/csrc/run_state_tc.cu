@@ -383,15 +383,15 @@ __global__ void __launch_bounds__(rst::kThreads, 1) run_state_tc_kernel(
 
 cudaError_t launch_run_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
                                 const float *dt_bias, float dt_min, float dt_max, float *slots, float *decays,
-                                int *status, bool reset_status, int B, int L, int H, int G, const RunLayout &lay,
-                                cudaStream_t st) {
+                                int *status, bool reset_status, int B, int L, int H, int G, int64_t x_row,
+                                int64_t bc_row, const RunLayout &lay, cudaStream_t st) {
     using namespace rst;
     CUtensorMap tm_x, tm_b, tm_s;
-    cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B,
-                                      (uint64_t)H * P * 2, (uint64_t)L * H * P * 2, 64, R, 1);
+    cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B, (uint64_t)x_row * 2,
+                                      (uint64_t)L * x_row * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16_3d(&tm_b, Bm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)G * N * 2,
-                          (uint64_t)L * G * N * 2, 64, R, 1);
+    e = make_tmap_bf16_3d(&tm_b, Bm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)bc_row * 2,
+                          (uint64_t)L * bc_row * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
     // every slot's two heads' S^T as rows of 64 fp32: boxes of 32 columns x 128 rows
     e = make_tmap_f32_2d(&tm_s, slots, (uint64_t)P, (uint64_t)lay.slots() * kPairHeads * N, (uint64_t)P * 4, 32, R);

@@ -39,7 +39,7 @@ def test_status_strings_and_version():
     for s in range(6):
         assert L.ssd_status_string(s)
     assert L.ssd_status_string(99) == b"unknown status"
-    assert L.ssd_abi_version() == 3
+    assert L.ssd_abi_version() == 4
     assert L.ssd_last_cuda_error() == 0
 
 
@@ -115,7 +115,8 @@ def prefill(**kw):
 
 
 @pytest.mark.parametrize("kw,want", [
-    (dict(x=None), INV), (dict(Bm=None), INV), (dict(y=None), INV), (dict(A_log=None), INV),
+    (dict(x=None), INV), (dict(Bm=None), INV), (dict(dt=None), INV), (dict(A_log=None), INV),
+    (dict(y=MIS), INV), (dict(Cm=None), INV),  # C is needed whenever y is (y = NULL: state only)
     (dict(x=MIS), INV), (dict(Cm=MIS), INV), (dict(h0=MIS), INV), (dict(D=MIS), INV),
     (dict(B=-1), INV), (dict(L=-3), INV), (dict(H=0), INV), (dict(G=3), INV), (dict(dtype=7), INV),
     (dict(dt_min=0.5, dt_max=0.1), INV), (dict(dt_min=-1.0), INV), (dict(dt_max=float("nan")), INV),
@@ -251,3 +252,37 @@ def test_header_is_plain_c_and_links(tmp_path):
                     f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
     assert out[0] == str(L.ssd_abi_version())
+
+
+def conv_prefill(**kw):
+    a = dict(xbc=A, w=A, b=None, dt=A, A_log=A, D=A, dt_bias=None, dt_min=1e-3, dt_max=0.1, h0=None,
+             y=A, h_final=A, cs=A, B=1, L=64, H=4, P=64, G=1, N=16, K=4, chunk=64, dtype=BF16, ws=A,
+             ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return L.ssd_conv_chunk_scan_fwd(a["xbc"], a["w"], a["b"], a["dt"], a["A_log"], a["D"], a["dt_bias"],
+                                     a["dt_min"], a["dt_max"], a["h0"], a["y"], a["h_final"], a["cs"], a["B"],
+                                     a["L"], a["H"], a["P"], a["G"], a["N"], a["K"], a["chunk"], a["dtype"],
+                                     a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(xbc=None), INV), (dict(w=None), INV), (dict(dt=None), INV), (dict(y=None), INV),
+    (dict(A_log=None), INV), (dict(xbc=MIS), INV), (dict(cs=MIS), INV), (dict(K=0), INV),
+    (dict(K=1), UNS), (dict(K=9), UNS), (dict(N=12, P=64), UNS), (dict(P=32), UNS), (dict(B=70000), UNS),
+    (dict(ws=None), WS), (dict(ws_bytes=4096), WS), (dict(G=3), INV), (dict(B=0), OK),
+])
+def test_conv_prefill_validation(kw, want):
+    assert conv_prefill(**kw) == want
+
+
+def test_conv_prefill_workspace_size():
+    # the prefill's own workspace, then the conv output [B, L, Cc] (256-byte aligned)
+    up = lambda v: -(-v // 256) * 256
+    for (B, Lx, H, P, G, N, K, chunk, dt) in [(1, 4096, 80, 64, 1, 128, 4, 256, BF16), (2, 300, 4, 64, 2, 16, 4, 64, F32),
+                                             (1, 0, 8, 64, 1, 128, 2, 256, BF16)]:
+        Cc = H * P + 2 * G * N
+        e = 2 if dt == BF16 else 4
+        got = L.ssd_conv_chunk_scan_workspace_size(B, Lx, H, P, G, N, K, chunk, dt)
+        assert got == L.ssd_chunk_scan_workspace_size(B, Lx, H, P, G, N, chunk, dt) + up(B * Lx * Cc * e)
+    assert L.ssd_conv_chunk_scan_workspace_size(1, 64, 4, 64, 1, 16, 9, 64, BF16) == 0   # K out of range
+    assert L.ssd_conv_chunk_scan_workspace_size(0, 64, 4, 64, 1, 16, 4, 64, BF16) == 0

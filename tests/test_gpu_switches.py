@@ -37,7 +37,8 @@ def test_without_programmatic_dependent_launch():
 
 def test_cuda_core_path_on_tensor_core_shapes():
     run_child({"SSD_PREFILL_KERNELS": "simt"},
-              [os.path.join(HERE, "test_gpu_prefill.py"), "-k", "m130m or m1p3b_b8 or sweep"])
+              [os.path.join(HERE, "test_gpu_prefill.py"), os.path.join(HERE, "test_gpu_conv_prefill.py"),
+               "-k", "m130m or m1p3b_b8 or sweep or conv_prefill"])
 
 
 def test_cuda_core_path_on_decay_edge_cases():
@@ -50,4 +51,4 @@ def test_fused_run_kernels():
     run_child({"SSD_PREFILL_KERNELS": "fused"},
               [os.path.join(HERE, "test_gpu_prefill.py"), os.path.join(HERE, "test_gpu_decay_edges.py"),
                os.path.join(HERE, "test_gpu_varlen.py"), os.path.join(HERE, "test_gpu_graph.py"),
-               "-k", "not decode"])
+               os.path.join(HERE, "test_gpu_conv_prefill.py"), "-k", "not decode or conv_prefill_then_decode"])
