@@ -264,12 +264,41 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
             for (int bi = 0; bi < 2; ++bi) {
                 const int cb = bi == 0 ? pc : 3 - pc;
                 if (cb > rq) continue;  // warp-uniform
+                const bool diag = cb == rq;
+                const bool factored = !diag || acs2[cb * 32] - acs2[cb * 32 + 31] <= kDiagFactorRange;
+                if (!factored) {
+                    // a diagonal sub-block whose decay spans more than fp32 can factor: each factor on
+                    // its own, 16 columns at a time (rare: only steep in-block decay takes it)
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const int c0 = cb * 32 + hf * 16;
+                        float v[16];
+                        tmem_ld16(tmem + lane_base + kColCB + c0, v);
+                        tmem_wait_ld();
+                        const float4 *a4 = reinterpret_cast<const float4 *>(acs2 + c0);
+                        const float4 *l4 = reinterpret_cast<const float4 *>(ldt + c0);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 a = a4[i], l = l4[i];
+                            v[4 * i + 0] *= ex2_approx((al - a.x) + l.x);
+                            v[4 * i + 1] *= ex2_approx((al - a.y) + l.y);
+                            v[4 * i + 2] *= ex2_approx((al - a.z) + l.z);
+                            v[4 * i + 3] *= ex2_approx((al - a.w) + l.w);
+                        }
+                        const int ld = myrow - c0;  // causal mask and the D skip, by select
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = i < ld ? v[i] : (i == ld ? v[i] + d : 0.f);
+                        uint32_t packed[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) packed[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                        tmem_st8(set + kOffPT + c0 / 2, packed);
+                    }
+                    continue;
+                }
                 float v[32];
                 tmem_ld16(tmem + lane_base + kColCB + cb * 32, *reinterpret_cast<float(*)[16]>(&v[0]));
                 tmem_ld16(tmem + lane_base + kColCB + cb * 32 + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
-                const bool diag = cb == rq;
-                const bool factored = !diag || acs2[cb * 32] - acs2[cb * 32 + 31] <= kDiagFactorRange;
-                if (factored) {
+                {
                     // P~_ls = CB_ls * 2^(acs2_l - ref) * 2^((ref - acs2_s) + ldt_s)
                     const float ref = diag ? acs2[cb * 32 + 15] : acs2[cb * 32 + 31];
                     vb[lane] = ex2_approx((ref - acs2[cb * 32 + lane]) + ldt[cb * 32 + lane]);
@@ -286,18 +315,6 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
                         v[4 * i + 3] *= u * c.w;
                     }
                     __syncwarp();
-                } else {
-                    tmem_wait_ld();
-                    const float4 *a4 = reinterpret_cast<const float4 *>(acs2 + cb * 32);
-                    const float4 *l4 = reinterpret_cast<const float4 *>(ldt + cb * 32);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 a = a4[i], l = l4[i];
-                        v[4 * i + 0] *= ex2_approx((al - a.x) + l.x);
-                        v[4 * i + 1] *= ex2_approx((al - a.y) + l.y);
-                        v[4 * i + 2] *= ex2_approx((al - a.z) + l.z);
-                        v[4 * i + 3] *= ex2_approx((al - a.w) + l.w);
-                    }
                 }
                 if (diag) {  // causal mask and the D skip; a select, so what lies above is dropped
                     const int ld = myrow - cb * 32;
