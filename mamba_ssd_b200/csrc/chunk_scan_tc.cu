@@ -152,6 +152,7 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
         if (lane == 0) {
+            const uint64_t release = l2_evict_first();  // x and h_prev^T: their last read, first to leave L2
             ItemCursor it(first, H, G, nk);
             int tiles = 0;
             for (int j = 0; j < cnt; ++j, it.next()) {
@@ -170,8 +171,9 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
                 uint8_t *st = stage(j);
                 const size_t row = ((size_t)it.b * H + h) * Lp + (size_t)it.k * R;
                 mbar_arrive_expect_tx(&st_full[s], 2 * kBox + 2 * R * 4);
-                tma_load_3d(st + kStX, &tm_x, h * P, it.k * R, it.b, &st_full[s]);
-                tma_load_2d(st + kStH, &tm_h, 0, (int)((((size_t)it.b * nk + it.k) * H + h) * N), &st_full[s]);
+                tma_load_3d_hint(st + kStX, &tm_x, h * P, it.k * R, it.b, &st_full[s], release);
+                tma_load_2d_hint(st + kStH, &tm_h, 0, (int)((((size_t)it.b * nk + it.k) * H + h) * N), &st_full[s],
+                                 release);
                 bulk_load(st + kStRows, dtf + row, R * 4, &st_full[s]);
                 bulk_load(st + kStRows + R * 4, acs + row, R * 4, &st_full[s]);
             }

@@ -146,6 +146,9 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
         if (lane == 0) {
+            // x is read once here: marked first to leave L2, so that the block states written
+            // meanwhile stay there for the state pass
+            const uint64_t stream_policy = l2_evict_first();
             ItemCursor it(first, H, G, nk);
             int tiles = 0;
             for (int j = 0; j < cnt; ++j, it.next()) {
@@ -161,7 +164,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
                 if (j >= kStages && !wait(&st_empty[s], ((j / kStages) - 1) & 1)) break;
                 uint8_t *st = stage(j);
                 mbar_arrive_expect_tx(&st_full[s], kBox);
-                tma_load_3d(st, &tm_x, h * P, it.k * R, it.b, &st_full[s]);
+                tma_load_3d_hint(st, &tm_x, h * P, it.k * R, it.b, &st_full[s], stream_policy);
             }
         }
     } else if (warp == 1) {

@@ -83,6 +83,15 @@ __device__ __forceinline__ T *after_wait(T *p) {
     return p;
 }
 
+// A global load with an L2 eviction-priority policy (a createpolicy result).
+__device__ __forceinline__ float4 ld_global_hint(const float4 *p, uint64_t policy) {
+    float4 v;
+    asm volatile("ld.global.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p), "l"(policy));
+    return v;
+}
+
 __host__ __device__ constexpr inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ constexpr inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 

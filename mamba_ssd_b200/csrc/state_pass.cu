@@ -17,6 +17,7 @@
 // The pass is HBM/L2 bound (it touches each chunk state twice).
 #include "common.cuh"
 #include "launch.h"
+#include "tc.cuh"
 
 namespace ssd {
 
@@ -90,13 +91,17 @@ __global__ void __launch_bounds__(256, 5) state_pass_t_kernel(const float *__res
     for (int i = 0; i < 4; ++i) s[i] = h0 ? h0[bh * PN + (size_t)(p0 + i) * N + n] : 0.f;
     const float *a_last = acs2 + bh * (size_t)nc * Q + (Q - 1);
     const size_t off = (size_t)n * P + p0;
+    // the block states' last read: marked first to leave L2, which keeps the h_prev^T just
+    // written there for the scan
+    const uint64_t release = tc::l2_evict_first();
     for (int c0 = 0; c0 < nc; c0 += kAhead) {
         float4 in[kAhead];
         float a[kAhead];
 #pragma unroll
         for (int j = 0; j < kAhead; ++j) {
             if (c0 + j < nc) {
-                in[j] = *reinterpret_cast<const float4 *>(statesT + (((size_t)b * nc + c0 + j) * H + h) * PN + off);
+                in[j] = ld_global_hint(reinterpret_cast<const float4 *>(statesT + (((size_t)b * nc + c0 + j) * H + h) * PN + off),
+                                       release);
                 a[j] = a_last[(size_t)(c0 + j) * Q];
             }
         }
