@@ -11,8 +11,9 @@ same run also measures the cached decode step of the 2.7B-shaped decode workload
 layers, ssm_state [B,80,64,128] fp32 + conv_state [B,5376,3] bf16, B in {1, 16}, 64
 steps from a state built by a 4096-token prefill) and reports it under "decode";
 "decode_vs_recompute" divides the prefill of a 1024-, 4096- and 16384-token prefix through
-the stack by one batch-1 decode step of it; "block_steps" times the prefix conv and the
-gated RMS norm on one 2.7B layer.
+the stack by one batch-1 decode step of it; "block_steps" times the prefix conv, the gated
+RMS norm and the conv-fed prefill on one 2.7B layer; "varlen" times a packed batch of 64
+sequences of 64 .. 4096 tokens in one varlen call against one prefill call per sequence.
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and
 torch.cuda.synchronize(), timed with CUDA events on the launching stream; the step is
@@ -143,7 +144,7 @@ KERNEL_METHOD_FLOPS = {"chunk_state": chunk_state_flops, "chunk_scan": chunk_sca
                        "run_state": chunk_state_flops, "chunk_scan_fused": chunk_scan_flops}
 # The sources a kernel's DRAM-traffic capture depends on: a capture is used only while these
 # files are byte-identical to the ones it was taken with.
-KERNEL_SOURCES = {"chunk_state": ["chunk_state_tc.cu", "items.cuh"], "state_pass": ["state_pass.cu"],
+KERNEL_SOURCES = {"chunk_state": ["chunk_state_tc.cu", "items.cuh"], "state_pass": ["state_pass.cu", "items.cuh"],
                   "chunk_scan": ["chunk_scan_tc.cu", "items.cuh"], "run_state": ["run_state_tc.cu", "runs.cuh"],
                   "run_pass": ["run_pass.cu", "runs.cuh"], "chunk_scan_fused": ["chunk_scan_fused.cu", "runs.cuh"]}
 SHARED_SOURCES = ["common.cuh", "tc.cuh", "launch.h", "tmap.cu"]
@@ -805,6 +806,70 @@ def bench_block_conv_prefill(torch, ssd, device, peaks, launches=16, buffers=8):
             "separate_note": "conv kernel, three torch copies splitting its output into x, B, C, then the prefill"}
 
 
+def bench_varlen(torch, ssd, device, reps=5):
+    """A packed varlen batch on the 2.7B layer shape (H = 80, P = 64, N = 128, bf16): the 64
+    sequences of 64 .. 4096 tokens of ssd_synth.varlen_lengths, each with its own h0, through
+    ssd_chunk_scan_varlen_fwd (one pass over all sequences' blocks), against the same work as
+    one ssd_chunk_scan_fwd call per sequence.  Each is captured in one graph and timed over
+    `reps` replays; the packed batch (0.5 GB of x in, 0.5 GB of y out) is larger than L2."""
+    import ssd_synth as S
+    H, P, G, N = PF["H"], PF["P"], PF["G"], PF["N"]
+    lengths = S.varlen_lengths()
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + n)
+    T, n_seq = cu[-1], len(lengths)
+    bf = torch.bfloat16
+    g = torch.Generator(device=device)
+    g.manual_seed(PF["seed"] + 83)
+    x = torch.randn((T, H, P), generator=g, device=device).to(bf)
+    dt = (torch.randn((T, H), generator=g, device=device) - 2.0).to(bf)
+    Bm = (torch.randn((T, G, N), generator=g, device=device) / math.sqrt(N)).to(bf)
+    Cm = (torch.randn((T, G, N), generator=g, device=device) / math.sqrt(N)).to(bf)
+    A_log = torch.log(torch.rand((H,), generator=g, device=device) * 15.0 + 1.0)
+    D = torch.randn((H,), generator=g, device=device)
+    h0 = torch.randn((n_seq, H, P, N), generator=g, device=device) * math.sqrt(0.1)
+    y = torch.empty_like(x)
+    hf = torch.empty_like(h0)
+    ws1 = torch.empty(ssd.ssd_chunk_scan_varlen_workspace_size(cu, H, P, G, N, PF["chunk"], bf), device=device,
+                      dtype=torch.uint8)
+    ws2 = torch.empty(ssd.ssd_chunk_scan_workspace_size(1, max(lengths), H, P, G, N, PF["chunk"], bf),
+                      device=device, dtype=torch.uint8)
+    kw = dict(D=D, chunk=PF["chunk"], dt_min=1e-3, dt_max=0.1)
+    stream = torch.cuda.Stream(device=device)
+    from mamba_ssd_b200 import _lib
+    lib = _lib.lib()
+
+    def one_pass():
+        ssd.ssd_chunk_scan_varlen_fwd(x, dt, A_log, Bm, Cm, cu, h0=h0, y=y, h_final=hf, workspace=ws1, **kw)
+
+    def per_sequence():
+        for i in range(n_seq):
+            a, b = cu[i], cu[i + 1]
+            ssd.ssd_chunk_scan_fwd(x[None, a:b], dt[None, a:b], A_log, Bm[None, a:b], Cm[None, a:b], h0=h0[i:i + 1],
+                                   y=y[None, a:b], h_final=hf[i:i + 1], workspace=ws2, **kw)
+
+    res = {}
+    for name, fn in (("one_pass", one_pass), ("per_sequence", per_sequence)):
+        with torch.cuda.stream(stream):
+            fn()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        n0 = lib.ssd_kernel_launch_count()
+        with torch.cuda.graph(graph, stream=stream):
+            fn()
+        launches = lib.ssd_kernel_launch_count() - n0
+        ms = time_graph(torch, graph, stream, reps)
+        res[name] = {"ms": ms, "tokens_per_s": T / (ms / 1e3), "launches": launches}
+        del graph
+    del x, dt, Bm, Cm, y
+    return {"workload": f"{n_seq} sequences of {min(lengths)}..{max(lengths)} tokens (log-uniform), {T} tokens, "
+                        f"H={H}, P={P}, N={N}, bf16, h0 per sequence",
+            "tokens": T, "sequences": n_seq, **res,
+            "speedup": res["per_sequence"]["ms"] / res["one_pass"]["ms"],
+            "per_sequence_note": "one ssd_chunk_scan_fwd call (three launches) per sequence, in one graph"}
+
+
 def time_graph(torch, graph, stream, reps):
     """Median CUDA-event time of `reps` replays of a captured graph, after one warm-up."""
     graph.replay()
@@ -1006,6 +1071,8 @@ def main():
                    "gated_rmsnorm": bench_block_norm(torch, ssd, device, peaks),
                    "conv_prefill": bench_block_conv_prefill(torch, ssd, device, peaks)}
     torch.cuda.empty_cache()
+    varlen = bench_varlen(torch, ssd, device)
+    torch.cuda.empty_cache()
 
     e2e = None
     if not args.no_e2e:  # every rank, the same collective steps in the same order
@@ -1033,7 +1100,7 @@ def main():
             "flops_per_layer_causal": prefill_flops_causal(B, L, H, P, G, N, Q),
             "roofline": roof, "kernels": kernels, "decode": decode, "e2e": e2e,
             "decode_vs_recompute": decode_vs_recompute(ms_step, decode, by_context),
-            "block_steps": block_steps,
+            "block_steps": block_steps, "varlen": varlen,
             "cpu_baseline": cpu, "clocks": pf["clocks"],
             "gpu_launches": pf["launches_per_step"] * args.steps,
             "peaks": peaks,

@@ -55,6 +55,8 @@
  * one call), ssd_segment_decay and ssd_state_combine (context-parallel prefill) added;
  * ssd_chunk_scan_fwd takes y = NULL (state only); ssd_chunk_scan_status(NULL) reads the
  * allocation-free entry's scratch.
+ * Version 5: ssd_chunk_scan_varlen_fwd runs a packed batch in one pass on the tensor-core
+ * path and takes its workspace size from the new ssd_chunk_scan_varlen_workspace_size.
  */
 #ifndef MAMBA_SSD_H
 #define MAMBA_SSD_H
@@ -202,18 +204,30 @@ SSD_API int ssd_state_combine(const float *states, const float *log2_decays, con
  *               sequences allowed: their h_final is their h0, or 0)
  *   h0, h_final [n_seq, H, P, N] float, each nullable
  *   A_log, D, dt_bias, dt_min, dt_max, chunk, dtype   as for ssd_chunk_scan_fwd
- *   workspace   ssd_chunk_scan_workspace_size(1, longest length, H, P, G, N, chunk, dtype)
- *               bytes, 256-byte aligned, shared by the sequences
- * Each sequence runs the prefill kernels of ssd_chunk_scan_fwd with B = 1, in order on
- * `stream` (three launches per non-empty sequence on the tensor-core path).  Everything is
- * validated before the first launch: SSD_ERR_INVALID_ARG for bad cu_seqlens or pointers,
- * SSD_ERR_UNSUPPORTED for a shape ssd_chunk_scan_fwd would not take or a sequence whose dt
- * rows would not start 16-byte aligned (never when H * sizeof(element) is a multiple of 16),
- * SSD_ERR_WORKSPACE.  A CUDA launch error stops the loop and is returned as SSD_ERR_CUDA.
- * The workspace's status word is reset once for the whole call (a 4-byte memset on `stream`)
- * and kept across the sequences: ssd_chunk_scan_status then reports SSD_ERR_TIMEOUT if any
- * sequence's bounded waits gave up.
+ *   workspace   ssd_chunk_scan_varlen_workspace_size(cu_seqlens, n_seq, H, P, G, N, chunk,
+ *               dtype) bytes, 256-byte aligned
+ * On the tensor-core path (bf16, P = 64, N = 128) the batch runs in one pass: a small kernel
+ * copies the table of its non-empty sequences (token start, first 128-token block, index)
+ * from cu_seqlens into the workspace, then the three prefill kernels walk every (sequence,
+ * block, head) item of the packed stream at once -- each sequence's blocks chained by the
+ * state pass from its own h0 to its own h_final, the rows after a sequence's end masked out of
+ * its last block -- so the launch count does not grow with n_seq.  An empty sequence's h_final
+ * is copied from h0 (or zeroed) on `stream`.  On the CUDA-core path (and with
+ * SSD_PREFILL_KERNELS=fused) each sequence runs the prefill kernels of ssd_chunk_scan_fwd with
+ * B = 1, in order on `stream`, sharing the workspace.  Everything is validated before the first
+ * launch: SSD_ERR_INVALID_ARG for bad cu_seqlens or pointers, SSD_ERR_UNSUPPORTED for a shape
+ * ssd_chunk_scan_fwd would not take or, on the per-sequence path, a sequence whose dt rows
+ * would not start 16-byte aligned (never when H * sizeof(element) is a multiple of 16),
+ * SSD_ERR_WORKSPACE.  A CUDA launch error is returned as SSD_ERR_CUDA.  The workspace's status
+ * word is this call's: ssd_chunk_scan_status reports SSD_ERR_TIMEOUT if any bounded wait of
+ * the call gave up.
+ *
+ * ssd_chunk_scan_varlen_workspace_size: the bytes ssd_chunk_scan_varlen_fwd needs for this
+ * batch (it grows with the total block count on the one-pass path), or 0 if n_seq <= 0 or an
+ * argument is invalid.
  */
+SSD_API size_t ssd_chunk_scan_varlen_workspace_size(const int *cu_seqlens, int n_seq, int H, int P, int G, int N,
+                                                    int chunk, int dtype);
 SSD_API int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float *A_log, const void *Bm,
                                       const void *Cm, const float *D, const float *dt_bias, float dt_min,
                                       float dt_max, const float *h0, void *y, float *h_final,
@@ -227,7 +241,7 @@ SSD_API int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float
  * outputs are then incomplete).  A NULL workspace reads the built-in scratch of
  * ssd_chunk_scan_fwd_noalloc on the current device, i.e. the status of the last
  * allocation-free call there.  For ssd_chunk_scan_varlen_fwd it is the status of the whole
- * call: SSD_ERR_TIMEOUT if any sequence's kernels timed out.  SSD_ERR_CUDA if the stream,
+ * call: SSD_ERR_TIMEOUT if any of its kernels timed out.  SSD_ERR_CUDA if the stream,
  * the copy or the scratch lookup failed.
  */
 SSD_API int ssd_chunk_scan_status(const void *workspace, void *stream);

@@ -8,12 +8,14 @@ the call raises ImportError.  There is no CPU or PyTorch fallback.  Build it wit
 from ._lib import SSDError, lib as load_library
 from .api import (decode_workspace, ssd_causal_conv1d_fwd, ssd_chunk_scan_fwd,
                   ssd_chunk_scan_fwd_noalloc, ssd_chunk_scan_status, ssd_chunk_scan_varlen_fwd,
-                  ssd_chunk_scan_workspace_size, ssd_conv_chunk_scan_fwd, ssd_conv_chunk_scan_workspace_size,
+                  ssd_chunk_scan_varlen_workspace_size, ssd_chunk_scan_workspace_size, ssd_conv_chunk_scan_fwd,
+                  ssd_conv_chunk_scan_workspace_size,
                   ssd_decode_status, ssd_decode_step, ssd_decode_workspace_size,
                   ssd_gated_rmsnorm_fwd, ssd_segment_decay, ssd_selftest_wait_timeout, ssd_state_combine)
 
 __all__ = ["SSDError", "load_library", "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_noalloc",
-           "ssd_chunk_scan_workspace_size", "ssd_chunk_scan_status", "ssd_decode_step",
+           "ssd_chunk_scan_workspace_size", "ssd_chunk_scan_varlen_workspace_size", "ssd_chunk_scan_status",
+           "ssd_decode_step",
            "ssd_decode_workspace_size", "ssd_decode_status", "decode_workspace", "ssd_causal_conv1d_fwd",
            "ssd_gated_rmsnorm_fwd", "ssd_selftest_wait_timeout", "ssd_chunk_scan_varlen_fwd",
            "ssd_conv_chunk_scan_fwd", "ssd_conv_chunk_scan_workspace_size", "ssd_segment_decay",

@@ -28,6 +28,7 @@ SIGNATURES = {
     "ssd_last_cuda_error": (_i, []),
     "ssd_abi_version": (_i, []),
     "ssd_chunk_scan_workspace_size": (_sz, [_i] * 8),
+    "ssd_chunk_scan_varlen_workspace_size": (_sz, [_vp] + [_i] * 7),
     "ssd_chunk_scan_fwd": (_i, [_vp, _vp, _fp, _vp, _vp, _fp, _fp, _f, _f, _fp, _vp, _fp]
                            + [_i] * 8 + [_vp, _sz, _vp]),
     "ssd_chunk_scan_status": (_i, [_vp, _vp]),

@@ -165,6 +165,15 @@ def ssd_state_combine(states, log2_decays, r, h0=None, out=None, stream=None):
     return out
 
 
+def ssd_chunk_scan_varlen_workspace_size(cu_seqlens, H, P, G, N, chunk=256, dtype=torch.bfloat16):
+    """Bytes of workspace ssd_chunk_scan_varlen_fwd needs for the batch cu_seqlens describes."""
+    import ctypes
+    cu = [int(v) for v in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    cu_arr = (ctypes.c_int * len(cu))(*cu)
+    return int(_lib.lib().ssd_chunk_scan_varlen_workspace_size(ctypes.cast(cu_arr, ctypes.c_void_p), len(cu) - 1,
+                                                               H, P, G, N, int(chunk), _DTYPES[dtype]))
+
+
 def ssd_chunk_scan_varlen_fwd(x, dt, A_log, Bm, Cm, cu_seqlens, D=None, chunk=256, h0=None,
                               dt_bias=None, dt_min=0.0, dt_max=math.inf, y=None, h_final=None,
                               workspace=None, want_h_final=True, stream=None):
@@ -193,11 +202,10 @@ def ssd_chunk_scan_varlen_fwd(x, dt, A_log, Bm, Cm, cu_seqlens, D=None, chunk=25
     if h_final is None and want_h_final:
         h_final = torch.empty((n, H, P, N), device=x.device, dtype=torch.float32)
     _need(h_final, "h_final", torch.float32, (n, H, P, N))
-    longest = max([b - a for a, b in zip(cu, cu[1:])] + [0])
-    need = _lib.lib().ssd_chunk_scan_workspace_size(1, longest, H, P, G, N, chunk, code)
-    if workspace is None:
-        workspace = torch.empty(max(need, 256), device=x.device, dtype=torch.uint8)
     cu_arr = (ctypes.c_int * len(cu))(*cu)
+    if workspace is None:
+        need = ssd_chunk_scan_varlen_workspace_size(cu, H, P, G, N, chunk, x.dtype)
+        workspace = torch.empty(max(need, 256), device=x.device, dtype=torch.uint8)
     s = _lib.lib().ssd_chunk_scan_varlen_fwd(
         _ptr(x), _ptr(dt), _ptr(A_log), _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(dt_bias),
         float(dt_min), float(dt_max), _ptr(h0), _ptr(y), _ptr(h_final), ctypes.cast(cu_arr, ctypes.c_void_p),

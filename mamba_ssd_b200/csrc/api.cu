@@ -224,6 +224,40 @@ size_t prefill_query_bytes(int B, int L, int H, int P, int G, int N, int chunk, 
     return need;
 }
 
+// A packed varlen batch: its non-empty sequences (m), their 128-token blocks in all, its
+// longest sequence.  Checks that the cumulative lengths start at 0 and never decrease.
+struct VarlenPlan {
+    int m = 0, nblocks = 0, max_len = 0;
+};
+int varlen_plan(const int *cu, int n_seq, VarlenPlan &p) {
+    if (cu[0] != 0) return SSD_ERR_INVALID_ARG;
+    p = VarlenPlan();
+    for (int i = 0; i < n_seq; ++i) {
+        if (cu[i + 1] < cu[i]) return SSD_ERR_INVALID_ARG;
+        const int len = cu[i + 1] - cu[i];
+        if (len > p.max_len) p.max_len = len;
+        if (len > 0) {
+            ++p.m;
+            p.nblocks += ssd::cdiv(len, ssd::kTcBlock);
+        }
+    }
+    return SSD_OK;
+}
+// The tensor-core path runs a packed batch in one pass; the CUDA-core and the run-carrying
+// kernels take its sequences one at a time.
+bool varlen_one_pass(int dtype, int P, int N) {
+    return use_tensor_cores() && !use_fused() && ssd::prefill_tc_supported(dtype, P, N);
+}
+// One pass: the block-major prefill workspace of all the batch's blocks, then the table
+// (tok0, blk0, seq: m + 1 ints each, each in its own 256-byte-aligned slot).
+size_t varlen_table_offset(const VarlenPlan &p, int H, int P, int N) {
+    return ssd::prefill_workspace_bytes(1, p.nblocks * ssd::kTcBlock, H, P, N, ssd::kTcBlock, true);
+}
+size_t varlen_query_bytes(const VarlenPlan &p, int H, int P, int G, int N, int chunk, int dtype) {
+    if (!varlen_one_pass(dtype, P, N)) return prefill_query_bytes(1, p.max_len, H, P, G, N, chunk, dtype);
+    return varlen_table_offset(p, H, P, N) + 3 * ssd::align_up(sizeof(int) * (size_t)(p.m + 1), 256);
+}
+
 }  // namespace
 
 extern "C" {
@@ -242,7 +276,7 @@ const char *ssd_status_string(int status) {
 
 int ssd_last_cuda_error(void) { return g_last_cuda_error; }
 
-int ssd_abi_version(void) { return 4; }
+int ssd_abi_version(void) { return 5; }
 
 size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, int N, int chunk,
                                      int dtype) {
@@ -259,6 +293,38 @@ namespace {
 // x_row, bc_row: elements between consecutive tokens of x and of B / C (H*P and G*N when
 // dense; Cc when x, B and C are views into one conv output [.., Cc]).  y == NULL computes the
 // state only (h_final), skipping the output kernels.
+// The tensor-core prefill's three launches over an equal-length batch (vl.n = 0: B sequences
+// of L tokens) or a packed varlen batch (B = 1, L = the packed token count, vl its table), with
+// nblocks 128-token blocks in all.
+int tc_prefill(const void *x, const void *dt, const float *A_log, const void *Bm, const void *Cm, const float *D,
+               const float *dt_bias, float dt_min, float dt_max, const float *h0, void *y, float *h_final, int B,
+               int L, int H, int P, int G, int N, const ssd::PrefillWorkspace &ws, const ssd::Varlen &vl, int nblocks,
+               bool reset_status, int64_t x_row, int64_t bc_row, cudaStream_t st) {
+    const int blk = ssd::kTcBlock;
+    cudaError_t e = cudaSuccess;
+    if (nblocks > 0) {
+        // the state kernel also forms the decay factors (step a1) of the items it owns
+        e = timed_launch(K_STATE, st, [&] {
+            return ssd::launch_chunk_state_tc(x, Bm, dt, A_log, dt_bias, dt_min, dt_max, ws.dtf, ws.acs, ws.states,
+                                              ws.status, reset_status, B, L, H, G, x_row, bc_row, vl, nblocks,
+                                              sm_count(), st);
+        });
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    e = timed_launch(K_PASS, st, [&] {
+        return ssd::launch_state_pass_t(ws.states, ws.acs, h0, h_final, ws.hT, B, L, H, P, N, blk, vl, nblocks, st);
+    });
+    if (e != cudaSuccess) return cuda_status(e);
+    if (nblocks > 0 && y) {
+        e = timed_launch(K_SCAN, st, [&] {
+            return ssd::launch_chunk_scan_tc(x, Bm, Cm, ws.dtf, ws.acs, ws.hT, D, y, ws.status, B, L, H, G, x_row,
+                                             bc_row, vl, nblocks, sm_count(), st);
+        });
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    return SSD_OK;
+}
+
 int prefill(const void *x, const void *dt, const float *A_log, const void *Bm, const void *Cm, const float *D,
             const float *dt_bias, float dt_min, float dt_max, const float *h0, void *y, float *h_final, int B, int L,
             int H, int P, int G, int N, int chunk, int dtype, void *workspace, size_t workspace_bytes, void *stream,
@@ -303,27 +369,9 @@ int prefill(const void *x, const void *dt, const float *A_log, const void *Bm, c
         // tensor-core path: 128-token blocks, block states in fp32, h_prev^T in bf16
         const int blk = ssd::kTcBlock;
         ssd::PrefillWorkspace ws = ssd::carve_prefill_workspace(workspace, B, L, H, P, N, blk, true);
-        if (L > 0) {
-            // the state kernel also forms the decay factors (step a1) of the items it owns
-            e = timed_launch(K_STATE, st, [&] {
-                return ssd::launch_chunk_state_tc(x, Bm, dt, A_log, dt_bias, dt_min, dt_max, ws.dtf, ws.acs,
-                                                  ws.states, ws.status, reset_status, B, L, H, G, x_row, bc_row,
-                                                  sm_count(), st);
-            });
-            if (e != cudaSuccess) return cuda_status(e);
-        }
-        e = timed_launch(K_PASS, st, [&] {
-            return ssd::launch_state_pass_t(ws.states, ws.acs, h0, h_final, ws.hT, B, L, H, P, N, blk, st);
-        });
-        if (e != cudaSuccess) return cuda_status(e);
-        if (L > 0 && want_y) {
-            e = timed_launch(K_SCAN, st, [&] {
-                return ssd::launch_chunk_scan_tc(x, Bm, Cm, ws.dtf, ws.acs, ws.hT, D, y, ws.status, B, L, H, G, x_row,
-                                                 bc_row, sm_count(), st);
-            });
-            if (e != cudaSuccess) return cuda_status(e);
-        }
-        return SSD_OK;
+        return tc_prefill(x, dt, A_log, Bm, Cm, D, dt_bias, dt_min, dt_max, h0, y, h_final, B, L, H, P, G, N,
+                          ws, ssd::Varlen{nullptr, nullptr, nullptr, 0}, B * ssd::cdiv(L, blk), reset_status, x_row,
+                          bc_row, st);
     }
     // CUDA-core path: the caller's chunk, fp32 throughout
     ssd::PrefillWorkspace ws = ssd::carve_prefill_workspace(workspace, B, L, H, P, N, chunk, false);
@@ -459,15 +507,10 @@ int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float *A_log,
                               int dtype, void *workspace, size_t workspace_bytes, void *stream) {
     if (n_seq < 0 || (n_seq > 0 && !cu_seqlens)) return SSD_ERR_INVALID_ARG;
     if (n_seq == 0) return SSD_OK;
-    // lengths: start at 0, never decrease
-    if (cu_seqlens[0] != 0) return SSD_ERR_INVALID_ARG;
-    int max_len = 0;
-    for (int i = 0; i < n_seq; ++i) {
-        const int len = cu_seqlens[i + 1] - cu_seqlens[i];
-        if (cu_seqlens[i + 1] < cu_seqlens[i]) return SSD_ERR_INVALID_ARG;
-        if (len > max_len) max_len = len;
-    }
-    int s = check_prefill_shape(1, max_len, H, P, G, N, chunk, dtype);
+    VarlenPlan plan;
+    int s = varlen_plan(cu_seqlens, n_seq, plan);
+    if (s != SSD_OK) return s;
+    s = check_prefill_shape(1, plan.max_len, H, P, G, N, chunk, dtype);
     if (s != SSD_OK) return s;
     if ((s = check_dt_range(dt_min, dt_max)) != SSD_OK) return s;
     const size_t e = dtype == SSD_DTYPE_BF16 ? 2 : 4;
@@ -478,21 +521,69 @@ int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float *A_log,
     if (any_tokens && (!x || !dt || !Bm || !Cm || !y || !aligned16(x) || !aligned16(dt) || !aligned16(Bm) ||
                        !aligned16(Cm) || !aligned16(y)))
         return SSD_ERR_INVALID_ARG;
-    // every sequence's rows must start on a 16-byte boundary (x, y, B, C always do for the
-    // supported P and N; dt does when H * e is a multiple of 16 or the offsets happen to be)
-    for (int i = 0; i < n_seq; ++i)
-        if (((size_t)cu_seqlens[i] * H * e) % 16 != 0 || ((size_t)cu_seqlens[i] * G * N * e) % 16 != 0)
-            return SSD_ERR_UNSUPPORTED;
-    const size_t need = prefill_query_bytes(1, max_len, H, P, G, N, chunk, dtype);
+    const bool one_pass = varlen_one_pass(dtype, P, N);
+    // the per-sequence path hands each sequence's rows to the prefill as its own arrays, which
+    // must start on a 16-byte boundary (x, y, B, C always do for the supported P and N; dt does
+    // when H * e is a multiple of 16 or the offsets happen to be)
+    if (!one_pass)
+        for (int i = 0; i < n_seq; ++i)
+            if (((size_t)cu_seqlens[i] * H * e) % 16 != 0 || ((size_t)cu_seqlens[i] * G * N * e) % 16 != 0)
+                return SSD_ERR_UNSUPPORTED;
+    const size_t need = varlen_query_bytes(plan, H, P, G, N, chunk, dtype);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return SSD_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t state = (size_t)H * P * N;
+    if (one_pass) {
+        // every argument is valid.  The empty sequences hand h0 (or zeros) straight through;
+        // the others run as one packed batch: the table of its non-empty sequences into the
+        // workspace, then the three tensor-core launches over all of their blocks.
+        cudaError_t ce = cudaSuccess;
+        for (int i = 0; i < n_seq && h_final; ++i) {
+            if (cu_seqlens[i + 1] != cu_seqlens[i]) continue;
+            ce = h0 ? cudaMemcpyAsync(h_final + i * state, h0 + i * state, state * sizeof(float),
+                                      cudaMemcpyDeviceToDevice, st)
+                    : cudaMemsetAsync(h_final + i * state, 0, state * sizeof(float), st);
+            if (ce != cudaSuccess) return cuda_status(ce);
+        }
+        ssd::PrefillWorkspace ws =
+            ssd::carve_prefill_workspace(workspace, 1, plan.nblocks * ssd::kTcBlock, H, P, N, ssd::kTcBlock, true);
+        if (plan.m == 0) {  // nothing to scan: the call's status word is still this call's
+            return cuda_status(cudaMemsetAsync(ws.status, 0, sizeof(int), st));
+        }
+        int *tab = reinterpret_cast<int *>(static_cast<char *>(workspace) + varlen_table_offset(plan, H, P, N));
+        const size_t slot = ssd::align_up(sizeof(int) * (size_t)(plan.m + 1), 256) / sizeof(int);
+        int *tok0 = tab, *blk0 = tab + slot, *seq = tab + 2 * slot;
+        ssd::VarlenTableChunk c;
+        c.base = c.count = 0;
+        int blocks = 0;
+        auto flush = [&]() -> cudaError_t {
+            cudaError_t r = c.count ? ssd::launch_varlen_table(c, tok0, blk0, seq, st) : cudaSuccess;
+            c.base += c.count;
+            c.count = 0;
+            return r;
+        };
+        for (int i = 0; i <= n_seq; ++i) {  // entries j = 0 .. m (the last one the end sentinel)
+            const bool end = i == n_seq;
+            if (!end && cu_seqlens[i + 1] == cu_seqlens[i]) continue;
+            c.tok0[c.count] = cu_seqlens[i];
+            c.blk0[c.count] = blocks;
+            c.seq[c.count] = end ? 0 : i;
+            ++c.count;
+            if (!end) blocks += ssd::cdiv(cu_seqlens[i + 1] - cu_seqlens[i], ssd::kTcBlock);
+            if (c.count == ssd::kVarlenChunk + 1 && (ce = flush()) != cudaSuccess) return cuda_status(ce);
+        }
+        if ((ce = flush()) != cudaSuccess) return cuda_status(ce);
+        const ssd::Varlen vl{tok0, blk0, seq, plan.m};
+        return tc_prefill(x, dt, A_log, Bm, Cm, D, dt_bias, dt_min, dt_max, h0, y, h_final, 1, cu_seqlens[n_seq], H,
+                          P, G, N, ws, vl, plan.nblocks, true, (int64_t)H * P, (int64_t)G * N, st);
+    }
     // every argument is valid: run each sequence through the prefill, in order on the stream,
     // sharing the workspace (each call's kernels start after the previous call's have ended).
     // The status word is reset once here and kept across the sequences, so that a timeout in
     // any of them is what ssd_chunk_scan_status reports for the call.
-    cudaError_t e0 = cudaMemsetAsync(workspace, 0, sizeof(int), static_cast<cudaStream_t>(stream));
+    cudaError_t e0 = cudaMemsetAsync(workspace, 0, sizeof(int), st);
     if (e0 != cudaSuccess) return cuda_status(e0);
-    const size_t state = (size_t)H * P * N;
     for (int i = 0; i < n_seq; ++i) {
         const size_t t0 = (size_t)cu_seqlens[i];
         const int len = cu_seqlens[i + 1] - cu_seqlens[i];
@@ -507,6 +598,15 @@ int ssd_chunk_scan_varlen_fwd(const void *x, const void *dt, const float *A_log,
         if (s != SSD_OK) return s;
     }
     return SSD_OK;
+}
+
+size_t ssd_chunk_scan_varlen_workspace_size(const int *cu_seqlens, int n_seq, int H, int P, int G, int N, int chunk,
+                                            int dtype) {
+    if (n_seq <= 0 || !cu_seqlens) return 0;
+    VarlenPlan plan;
+    if (varlen_plan(cu_seqlens, n_seq, plan) != SSD_OK) return 0;
+    if (check_prefill_shape(1, plan.max_len, H, P, G, N, chunk, dtype) != SSD_OK) return 0;
+    return varlen_query_bytes(plan, H, P, G, N, chunk, dtype);
 }
 
 int ssd_chunk_scan_status(const void *workspace, void *stream) {

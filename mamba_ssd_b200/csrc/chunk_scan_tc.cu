@@ -32,15 +32,20 @@
 // otherwise its factors are taken one by one.  Above the diagonal P~ is zero: those TMEM
 // columns are cleared once per CTA and never written again.
 //
-// Structure: persistent CTAs own contiguous ranges of items ordered (batch, block, head), so
-// consecutive items share the C/B tiles and CB.  Warp-specialised, every role with its own
+// Structure: persistent CTAs own contiguous ranges of items ordered (sequence, block, head) of
+// an equal-length or a packed varlen batch (items.cuh), so consecutive items share the C/B
+// tiles and CB.  Warp-specialised, every role with its own
 // loop, the roles meeting only at mbarriers:
 //   warp 0       TMA producer: C/B tiles per (batch, block, group); x tile, h_prev^T tile and
 //                the item's per-token factors into a ring of kStages stages
 //   warp 1       MMA issuer (one lane): CB per tile; O and Y per item into one of two TMEM sets
 //   warps 2..9   P~ of an item into its TMEM set
 //   warps 10..17 epilogue: y = Y + exp(acs) O of an item into a swizzled shared-memory tile
-//                that one TMA store writes out (tokens past L are clipped by the store)
+//                that one TMA store writes out (tokens past L are clipped by the store); the
+//                ragged last block of a packed varlen sequence is stored row by row instead,
+//                its real rows only, since the rows after it belong to the next sequence
+//                (their P~ rows only ever meet x rows after the sequence's end through the
+//                causal mask's zeros, so they cannot reach a real row)
 // so the tensor core runs item j's products while P~ of item j+1 is formed and item j-1's
 // outputs are written.
 #include "common.cuh"
@@ -73,11 +78,13 @@ constexpr float kDiagFactorRange = 96.f;  // log2 range of a diagonal sub-block 
 constexpr int kEpiBar = 1;                 // named barrier of the epilogue warps
 }  // namespace csc
 
+template <bool VARLEN>
 __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_h,
     const __grid_constant__ CUtensorMap tm_y, const float *__restrict__ dtf, const float *__restrict__ acs,
-    const float *__restrict__ D, int *__restrict__ status, int H, int G, int nk, int total) {
+    const float *__restrict__ D, __nv_bfloat16 *__restrict__ y, int *__restrict__ status, int L, int H, int G,
+    int nk, int total, const Varlen vl) {
     using namespace csc;
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
@@ -100,7 +107,7 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
     const int first = (int)((long long)blockIdx.x * total / gridDim.x);
     const int cnt = (int)((long long)(blockIdx.x + 1) * total / gridDim.x) - first;
     if (cnt <= 0) return;
-    const size_t Lp = (size_t)nk * R;
+    const int nblk = total / H;  // blocks of the whole batch
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -135,7 +142,9 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
     dtf = after_wait(dtf);
     acs = after_wait(acs);
     D = after_wait(D);
+    y = after_wait(y);
     status = after_wait(status);
+    const Varlen tab = {after_wait(vl.tok0), after_wait(vl.blk0), after_wait(vl.seq), vl.n};
 
     auto stage = [&](int j) { return smem + kOffStage + (uint32_t)(j % kStages) * kStageBytes; };
     // a bounded wait that gives up at once when another role has already timed out
@@ -153,27 +162,26 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
         // ---------------------------------------------------------------- producer
         if (lane == 0) {
             const uint64_t release = l2_evict_first();  // x and h_prev^T: their last read, first to leave L2
-            ItemCursor it(first, H, G, nk);
+            ItemCursor<VARLEN> it(first, H, G, nk, L, tab);
             int tiles = 0;
             for (int j = 0; j < cnt; ++j, it.next()) {
                 const int h = it.h();
                 if (j == 0 || it.tile_first()) {
                     if (tiles > 0 && !wait(ld_empty, (tiles - 1) & 1)) break;
                     mbar_arrive_expect_tx(ld_full, 4 * kBox);
-                    tma_load_3d(smem + kOffC, &tm_c, it.g * N, it.k * R, it.b, ld_full);
-                    tma_load_3d(smem + kOffC + kBox, &tm_c, it.g * N + 64, it.k * R, it.b, ld_full);
-                    tma_load_3d(smem + kOffB, &tm_b, it.g * N, it.k * R, it.b, ld_full);
-                    tma_load_3d(smem + kOffB + kBox, &tm_b, it.g * N + 64, it.k * R, it.b, ld_full);
+                    tma_load_3d(smem + kOffC, &tm_c, it.g * N, it.row(), it.zb, ld_full);
+                    tma_load_3d(smem + kOffC + kBox, &tm_c, it.g * N + 64, it.row(), it.zb, ld_full);
+                    tma_load_3d(smem + kOffB, &tm_b, it.g * N, it.row(), it.zb, ld_full);
+                    tma_load_3d(smem + kOffB + kBox, &tm_b, it.g * N + 64, it.row(), it.zb, ld_full);
                     ++tiles;
                 }
                 const int s = j % kStages;
                 if (j >= kStages && !wait(&st_empty[s], ((j / kStages) - 1) & 1)) break;
                 uint8_t *st = stage(j);
-                const size_t row = ((size_t)it.b * H + h) * Lp + (size_t)it.k * R;
+                const size_t row = ((size_t)h * nblk + it.gblk()) * R;  // head-major factor rows
                 mbar_arrive_expect_tx(&st_full[s], 2 * kBox + 2 * R * 4);
-                tma_load_3d_hint(st + kStX, &tm_x, h * P, it.k * R, it.b, &st_full[s], release);
-                tma_load_2d_hint(st + kStH, &tm_h, 0, (int)((((size_t)it.b * nk + it.k) * H + h) * N), &st_full[s],
-                                 release);
+                tma_load_3d_hint(st + kStX, &tm_x, h * P, it.row(), it.zb, &st_full[s], release);
+                tma_load_2d_hint(st + kStH, &tm_h, 0, (int)(((size_t)it.gblk() * H + h) * N), &st_full[s], release);
                 bulk_load(st + kStRows, dtf + row, R * 4, &st_full[s]);
                 bulk_load(st + kStRows + R * 4, acs + row, R * 4, &st_full[s]);
             }
@@ -185,7 +193,7 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
             constexpr uint32_t id_kmn = idesc_bf16_f32(128, 64, false, true);  // K-major A, MN-major B
             const uint64_t dc = desc_kmajor_sw128(smem_u32(smem + kOffC));
             const uint64_t db = desc_kmajor_sw128(smem_u32(smem + kOffB));
-            ItemCursor it(first, H, G, nk);
+            ItemCursor<VARLEN> it(first, H, G, nk, L, tab);
             int tiles = 0;
             for (int j = 0; j < cnt; ++j, it.next()) {
                 const int s = j % kStages, t = j & 1;
@@ -244,7 +252,7 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
                     if (cb > rq) tmem_st16(tmem + lane_base + kSet0 + t * kSet + kOffPT + cb * 16, zero);
                 }
         }
-        ItemCursor it(first, H, G, nk);
+        ItemCursor<VARLEN> it(first, H, G, nk, L, tab);
         int tiles = 0;
         for (int j = 0; j < cnt; ++j, it.next()) {
             const int s = j % kStages, t = j & 1;
@@ -342,11 +350,14 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
         const int myrow = rq * 32 + lane;
         const uint32_t lane_base = (uint32_t)(rq * 32) << 16;
         const bool leader = warp == 2 + kPt && lane == 0;  // issues the stores
-        ItemCursor it(first, H, G, nk);
+        ItemCursor<VARLEN> it(first, H, G, nk, L, tab);
         for (int j = 0; j < cnt; ++j, it.next()) {
             const int t = j & 1, h = it.h();
             // exp(acs_l) from the log2-form cumsum; read here, the stage may be refilled by now
-            const float al = __ldg(acs + ((size_t)it.b * H + h) * Lp + (size_t)it.k * R + myrow);
+            const float al = __ldg(acs + ((size_t)h * nblk + it.gblk()) * R + myrow);
+            // a packed sequence's ragged last block: the rows after its end belong to the next
+            // sequence, so its real rows are stored directly instead of by the tile store
+            const int direct = VARLEN ? it.valid() : R;
             const bool ok = __all_sync(0xffffffffu, wait(&acc_full[t], (j >> 1) & 1));
             uint32_t o[16];
             if (ok) {
@@ -369,6 +380,15 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
             // the staging tile is free once the previous item's store has read it
             if (leader) bulk_wait_read();
             if (!named_barrier_and(kEpiBar, kEpi * 32, ok)) break;
+            if (direct < R) {  // item-uniform
+                if (myrow < direct) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(y + ((size_t)it.row() + myrow) * H * P + (size_t)h * P +
+                                                           half * 32);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+                }
+                continue;
+            }
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 *reinterpret_cast<uint4 *>(smem + kOffOut + sw128_offset(myrow, half * 4 + q)) =
@@ -376,7 +396,7 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
             fence_proxy_async_smem();
             named_barrier(kEpiBar, kEpi * 32);
             if (leader) {
-                tma_store_3d(&tm_y, smem + kOffOut, h * P, it.k * R, it.b);
+                tma_store_3d(&tm_y, smem + kOffOut, h * P, it.row(), it.zb);
                 bulk_commit();
             }
         }
@@ -398,11 +418,11 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
 
 cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, const float *dtf,
                                  const float *acs, const __nv_bfloat16 *hT, const float *D, void *y,
-                                 int *status, int B, int L, int H, int G, int64_t x_row, int64_t bc_row, int num_sms,
-                                 cudaStream_t st) {
+                                 int *status, int B, int L, int H, int G, int64_t x_row, int64_t bc_row,
+                                 const Varlen &vl, int nblocks, int num_sms, cudaStream_t st) {
     using namespace csc;
-    const int nk = cdiv(L, R);
-    const int total = B * nk * H;
+    const int nk = cdiv(L, R);  // blocks per sequence of an equal-length batch
+    const int total = nblocks * H;
     CUtensorMap tm_x, tm_b, tm_c, tm_h, tm_y;
     // x, B and C rows are x_row and bc_row elements apart (H*P and G*N when dense); y is dense
     cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B, (uint64_t)x_row * 2,
@@ -414,16 +434,20 @@ cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, 
     e = make_tmap_bf16_3d(&tm_c, Cm, (uint64_t)G * N, (uint64_t)L, (uint64_t)B, (uint64_t)bc_row * 2,
                           (uint64_t)L * bc_row * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16_2d(&tm_h, hT, (uint64_t)P, (uint64_t)B * nk * H * N, (uint64_t)P * 2, 64, R);
+    e = make_tmap_bf16_2d(&tm_h, hT, (uint64_t)P, (uint64_t)nblocks * H * N, (uint64_t)P * 2, 64, R);
     if (e != cudaSuccess) return e;
     e = make_tmap_bf16_3d(&tm_y, y, (uint64_t)H * P, (uint64_t)L, (uint64_t)B, (uint64_t)H * P * 2,
                           (uint64_t)L * H * P * 2, 64, R, 1);
     if (e != cudaSuccess) return e;
     const int grid = total < num_sms ? total : num_sms;
-    e = raise_smem_limit<chunk_scan_tc_kernel>((int)kSmem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(chunk_scan_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, tm_x, tm_b, tm_c, tm_h, tm_y,
-                      dtf, acs, D, status, H, G, nk, total);
+    auto launch = [&](auto tag) {
+        constexpr auto kernel = decltype(tag)::kernel;
+        cudaError_t r = raise_smem_limit<kernel>((int)kSmem);
+        if (r != cudaSuccess) return r;
+        return launch_pdl(kernel, dim3(grid), dim3(kThreads), kSmem, st, tm_x, tm_b, tm_c, tm_h, tm_y, dtf, acs, D,
+                          (__nv_bfloat16 *)y, status, L, H, G, nk, total, vl);
+    };
+    return vl.n ? launch(KernelTag<chunk_scan_tc_kernel<true>>{}) : launch(KernelTag<chunk_scan_tc_kernel<false>>{});
 }
 
 }  // namespace ssd

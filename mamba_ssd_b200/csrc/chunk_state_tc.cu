@@ -27,11 +27,14 @@
 // taken before log2(dt) is added: folded into one number, log2(dt) would be lost to rounding
 // once |acs2| is large (a decay of many nats per token).  Source: the
 // blog walk-through's §1.1 (discretisation, chunked cumulative decay) and §1.2 (the fused
-// softplus -> clip -> exp chain); §4.1 (the decay in float32).  Tokens past L get dt = 0, so
-// their decay is 1 and their weight exactly 0 (ldt = -inf).
+// softplus -> clip -> exp chain); §4.1 (the decay in float32).  Tokens past the end of their
+// sequence get dt = 0, so their decay is 1 and their weight exactly 0 (ldt = -inf): in a packed
+// varlen batch the x and B rows after a sequence's end, which belong to the next sequence, drop
+// out of its last block's state that way.
 //
-// Structure: persistent CTAs, one per SM, each owning a contiguous range of (batch, block,
-// head) items (consecutive items share the block's B tile).  Warp-specialised:
+// Structure: persistent CTAs, one per SM, each owning a contiguous range of (sequence, block,
+// head) items of an equal-length or a packed varlen batch (items.cuh; consecutive items share
+// the block's B tile).  Warp-specialised:
 //   warp 0       TMA producer: B tile per (batch, block, group); x tile per item into a ring
 //                of kStages stages
 //   warps 18..21 decay factors of an item into its stage and to global memory (warp 18 + s
@@ -68,11 +71,13 @@ constexpr uint32_t kSmem = kOffBar + 256 + 1024;  // + slack for 1024-byte align
 constexpr uint32_t kTmemCols = 256;               // two 128-column fp32 accumulators [hi | lo]
 }  // namespace cst
 
+template <bool VARLEN>
 __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_s, const __nv_bfloat16 *__restrict__ dt, const float *__restrict__ A_log,
     const float *__restrict__ dt_bias, float dt_min, float dt_max, float *__restrict__ dtf,
-    float *__restrict__ acs, int *__restrict__ status, int reset_status, int L, int H, int G, int nk, int total) {
+    float *__restrict__ acs, int *__restrict__ status, int reset_status, int L, int H, int G, int nk, int total,
+    const Varlen vl) {
     using namespace cst;
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
@@ -93,7 +98,6 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     const int first = (int)((long long)blockIdx.x * total / gridDim.x);
     const int cnt = (int)((long long)(blockIdx.x + 1) * total / gridDim.x) - first;
     if (cnt <= 0) return;
-    const size_t Lp = (size_t)nk * R;
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -127,6 +131,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     dtf = after_wait(dtf);
     acs = after_wait(acs);
     status = after_wait(status);
+    const Varlen tab = {after_wait(vl.tok0), after_wait(vl.blk0), after_wait(vl.seq), vl.n};
     // this call's status word starts clean (a later wait of the call may record a timeout),
     // unless the caller keeps one word across several calls (the varlen prefill)
     if (reset_status && blockIdx.x == 0 && tid == 0) *status = SSD_OK;
@@ -149,22 +154,22 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
             // x is read once here: marked first to leave L2, so that the block states written
             // meanwhile stay there for the state pass
             const uint64_t stream_policy = l2_evict_first();
-            ItemCursor it(first, H, G, nk);
+            ItemCursor<VARLEN> it(first, H, G, nk, L, tab);
             int tiles = 0;
             for (int j = 0; j < cnt; ++j, it.next()) {
                 const int h = it.h();
                 if (j == 0 || it.tile_first()) {
                     if (tiles > 0 && !wait(b_empty, (tiles - 1) & 1)) break;
                     mbar_arrive_expect_tx(b_full, 2 * kBox);
-                    tma_load_3d(smem + kOffB, &tm_b, it.g * N, it.k * R, it.b, b_full);
-                    tma_load_3d(smem + kOffB + kBox, &tm_b, it.g * N + 64, it.k * R, it.b, b_full);
+                    tma_load_3d(smem + kOffB, &tm_b, it.g * N, it.row(), it.zb, b_full);
+                    tma_load_3d(smem + kOffB + kBox, &tm_b, it.g * N + 64, it.row(), it.zb, b_full);
                     ++tiles;
                 }
                 const int s = j % kStages;
                 if (j >= kStages && !wait(&st_empty[s], ((j / kStages) - 1) & 1)) break;
                 uint8_t *st = stage(j);
                 mbar_arrive_expect_tx(&st_full[s], kBox);
-                tma_load_3d_hint(st, &tm_x, h * P, it.k * R, it.b, &st_full[s], stream_policy);
+                tma_load_3d_hint(st, &tm_x, h * P, it.row(), it.zb, &st_full[s], stream_policy);
             }
         }
     } else if (warp == 1) {
@@ -172,7 +177,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(128, 128, true, true);  // N = [hi | lo]
             const uint64_t da = desc_mnmajor_sw128(smem_u32(smem + kOffB), kBox);
-            ItemCursor it(first, H, G, nk);
+            ItemCursor<VARLEN> it(first, H, G, nk, L, tab);
             int tiles = 0;
             for (int j = 0; j < cnt; ++j, it.next()) {
                 const int s = j % kStages, a = j & 1;
@@ -203,21 +208,22 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
         // stand-alone decay kernel, so both give the same bits).  The strided dt loads of the
         // next item are issued before this one is processed.
         const int s = warp - kPrepWarp;
-        auto load_raw = [&](const ItemCursor &c, float (&r)[4]) {
-            const int t0 = c.k * R + lane * 4, h = c.h();
+        auto load_raw = [&](const ItemCursor<VARLEN> &c, float (&r)[4]) {
+            const int t0 = c.k * R + lane * 4, h = c.h();  // t0: token of the sequence
+            const size_t row = (size_t)c.zb * L + c.row0 + t0;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                r[i] = t0 + i < L ? __bfloat162float(dt[((size_t)c.b * L + t0 + i) * H + h]) : 0.f;
+                r[i] = t0 + i < c.len ? __bfloat162float(dt[(row + i) * H + h]) : 0.f;
         };
-        auto step = [&](ItemCursor &c) {
+        auto step = [&](ItemCursor<VARLEN> &c) {
 #pragma unroll
             for (int i = 0; i < kStages; ++i) c.next();
         };
-        auto load_par = [&](const ItemCursor &c, float &bias, float &alog) {
+        auto load_par = [&](const ItemCursor<VARLEN> &c, float &bias, float &alog) {
             bias = dt_bias ? __ldg(dt_bias + c.h()) : 0.f;
             alog = __ldg(A_log + c.h());
         };
-        ItemCursor it(first + s, H, G, nk), ahead(first + s, H, G, nk);
+        ItemCursor<VARLEN> it(first + s, H, G, nk, L, tab), ahead(first + s, H, G, nk, L, tab);
         float r0[4] = {0.f, 0.f, 0.f, 0.f}, b0 = 0.f, l0 = 0.f;
         if (s < cnt) {
             load_raw(ahead, r0);
@@ -238,7 +244,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
             float d[4], run = 0.f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                d[i] = t0 + i < L ? discretise_dt(r0[i], bias, dt_min, dt_max) : 0.f;
+                d[i] = t0 + i < it.len ? discretise_dt(r0[i], bias, dt_min, dt_max) : 0.f;
                 run += d[i] * A;
             }
             float acc = warp_inclusive_sum(run) - run;  // exclusive prefix of this lane
@@ -252,7 +258,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
             // a ragged last block: the padded slots take exactly the last real token's cumsum
             // (the lanes' partial sums round differently; the block's end must stand for that
             // token, so that its own weight exp2(acs2_end - acs2_last) is exactly 1)
-            const int tl = L - 1 - it.k * R;  // slot of the last real token
+            const int tl = it.len - 1 - it.k * R;  // slot of the last real token
             if (tl < R - 1) {                 // warp-uniform
                 const float mine = (tl >> 2) == lane ? ((tl & 3) == 0 ? a2[0] : (tl & 3) == 1 ? a2[1]
                                                         : (tl & 3) == 2 ? a2[2] : a2[3]) : 0.f;
@@ -266,7 +272,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
             float *rows = reinterpret_cast<float *>(stage(j) + 2 * kBox);
             reinterpret_cast<float4 *>(rows)[lane] = c4;
             reinterpret_cast<float4 *>(rows + R)[lane] = a4;
-            const size_t g = ((size_t)it.b * H + h) * Lp + (size_t)t0;
+            const size_t g = ((size_t)h * (total / H) + it.gblk()) * R + (size_t)lane * 4;  // head-major rows
             *reinterpret_cast<float4 *>(dtf + g) = c4;
             *reinterpret_cast<float4 *>(acs + g) = a4;
             __syncwarp();
@@ -326,7 +332,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
         const int n = quarter * 32 + lane;
         const bool leader = warp == 2 + kXform && lane == 0;  // issues the stores
         uint8_t *box = smem + kOffOut + half * kBox;
-        ItemCursor it(first, H, G, nk);
+        ItemCursor<VARLEN> it(first, H, G, nk, L, tab);
         for (int j = 0; j < cnt; ++j, it.next()) {
             const int a = j & 1;
             const bool ok = __all_sync(0xffffffffu, wait(&acc_full[a], (j >> 1) & 1));
@@ -357,7 +363,7 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
             fence_proxy_async_smem();
             named_barrier(kEpiBar, kEpi * 32);
             if (leader) {
-                const int row = (int)((((size_t)it.b * nk + it.k) * H + it.h()) * N);
+                const int row = (int)(((size_t)it.gblk() * H + it.h()) * N);
                 tma_store_2d(&tm_s, smem + kOffOut, 0, row);
                 tma_store_2d(&tm_s, smem + kOffOut + kBox, 32, row);
                 bulk_commit();
@@ -386,10 +392,11 @@ bool prefill_tc_supported(int dtype, int P, int N) {
 cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
                                   const float *dt_bias, float dt_min, float dt_max, float *dtf, float *acs,
                                   float *states, int *status, bool reset_status, int B, int L, int H, int G,
-                                  int64_t x_row, int64_t bc_row, int num_sms, cudaStream_t st) {
+                                  int64_t x_row, int64_t bc_row, const Varlen &vl, int nblocks, int num_sms,
+                                  cudaStream_t st) {
     using namespace cst;
-    const int nk = cdiv(L, R);
-    const int total = B * nk * H;
+    const int nk = cdiv(L, R);  // blocks per sequence of an equal-length batch
+    const int total = nblocks * H;
     CUtensorMap tm_x, tm_b, tm_s;
     // x and B rows are x_row and bc_row elements apart (H*P and G*N when dense)
     cudaError_t e = make_tmap_bf16_3d(&tm_x, x, (uint64_t)H * P, (uint64_t)L, (uint64_t)B, (uint64_t)x_row * 2,
@@ -402,11 +409,14 @@ cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const void *dt,
     e = make_tmap_f32_2d(&tm_s, states, (uint64_t)P, (uint64_t)total * N, (uint64_t)P * 4, 32, R);
     if (e != cudaSuccess) return e;
     const int grid = total < num_sms ? total : num_sms;
-    e = raise_smem_limit<chunk_state_tc_kernel>((int)kSmem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(chunk_state_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, tm_x, tm_b, tm_s,
-                      (const __nv_bfloat16 *)dt, A_log, dt_bias, dt_min, dt_max, dtf, acs, status, reset_status ? 1 : 0, L, H, G, nk,
-                      total);
+    auto launch = [&](auto tag) {
+        constexpr auto kernel = decltype(tag)::kernel;
+        cudaError_t r = raise_smem_limit<kernel>((int)kSmem);
+        if (r != cudaSuccess) return r;
+        return launch_pdl(kernel, dim3(grid), dim3(kThreads), kSmem, st, tm_x, tm_b, tm_s, (const __nv_bfloat16 *)dt,
+                          A_log, dt_bias, dt_min, dt_max, dtf, acs, status, reset_status ? 1 : 0, L, H, G, nk, total, vl);
+    };
+    return vl.n ? launch(KernelTag<chunk_state_tc_kernel<true>>{}) : launch(KernelTag<chunk_state_tc_kernel<false>>{});
 }
 
 }  // namespace ssd

@@ -8,6 +8,7 @@
 
 #include <atomic>
 
+#include "items.cuh"
 #include "runs.cuh"
 
 namespace ssd {
@@ -26,6 +27,12 @@ cudaError_t raise_smem_limit(int bytes) {
     if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
     return e;
 }
+
+// A kernel as a type, for generic lambdas that launch one of several instantiations.
+template <auto K>
+struct KernelTag {
+    static constexpr auto kernel = K;
+};
 
 // Launches of the tensor-core prefill kernels use programmatic stream serialization (each may
 // be scheduled while the kernel before it finishes; the kernels order every global access
@@ -50,9 +57,10 @@ cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t 
 // Prefill workspace layout, 256-byte aligned pieces:
 //   status int32 (256-byte slot): SSD_OK, or SSD_ERR_TIMEOUT if a bounded wait gave up
 //   dtf    [B][H][Lp]          clipped dt per token (0 past the end of the sequence); on the
-//                              tensor-core path its base-2 logarithm, log2(dt), instead
+//                              tensor-core path its base-2 logarithm, log2(dt), instead, as
+//                              [H][B*nb][128] (each head's blocks of the whole batch in a row)
 //   acs    [B][H][Lp]          inclusive cumsum of dt*A inside each block; on the tensor-core
-//                              path acs2 = that cumsum times log2(e)
+//                              path acs2 = that cumsum times log2(e), laid out like dtf
 //   states [B][nb][H][P][N]    fp32 block states; the CUDA-core path overwrites them in
 //                              place with the state each block starts from (h_prev); the
 //                              tensor-core path stores each transposed, [N][P]
@@ -81,18 +89,32 @@ constexpr int kTcBlock = 128;
 bool prefill_tc_supported(int dtype, int P, int N);
 // chunk_state_tc also forms the log2-form decay factors (dtf = log2(dt), acs = acs2) from dt and
 // resets the status word: it is the first kernel of a tensor-core prefill call.
+// Their workspace (global block gb, head h: factor rows at (h*nblocks + gb)*128, states at
+// (gb*H + h)*P*N), for an equal-length batch (B sequences of L tokens, nblocks = B*ceil(L/128),
+// vl.n = 0) or a packed varlen batch (B = 1, L = the packed token count, vl = the non-empty
+// sequences' table, nblocks = its block count).
 cudaError_t launch_chunk_state_tc(const void *x, const void *Bm, const void *dt, const float *A_log,
                                   const float *dt_bias, float dt_min, float dt_max, float *dtf, float *acs,
                                   float *states, int *status, bool reset_status, int B, int L, int H, int G,
-                                  int64_t x_row, int64_t bc_row, int num_sms, cudaStream_t st);
+                                  int64_t x_row, int64_t bc_row, const Varlen &vl, int nblocks, int num_sms,
+                                  cudaStream_t st);
 
 cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, const float *dtf,
                                  const float *acs, const __nv_bfloat16 *hT, const float *D, void *y,
-                                 int *status, int B, int L, int H, int G, int64_t x_row, int64_t bc_row, int num_sms,
-                                 cudaStream_t st);
+                                 int *status, int B, int L, int H, int G, int64_t x_row, int64_t bc_row,
+                                 const Varlen &vl, int nblocks, int num_sms, cudaStream_t st);
 cudaError_t launch_state_pass_t(const float *states, const float *acs, const float *h0, float *h_final,
-                                __nv_bfloat16 *hT, int B, int L, int H, int P, int N, int chunk,
-                                cudaStream_t st);
+                                __nv_bfloat16 *hT, int B, int L, int H, int P, int N, int chunk, const Varlen &vl,
+                                int nblocks, cudaStream_t st);
+
+// Up to kVarlenChunk entries of a packed varlen batch's table, written at [base, base + count)
+// of the workspace copy by one launch.
+constexpr int kVarlenChunk = 256;
+struct VarlenTableChunk {
+    int base, count;
+    int tok0[kVarlenChunk + 1], blk0[kVarlenChunk + 1], seq[kVarlenChunk + 1];
+};
+cudaError_t launch_varlen_table(const VarlenTableChunk &c, int *tok0, int *blk0, int *seq, cudaStream_t st);
 
 // Fused tensor-core prefill (bf16 storage, P = 64, N = 128, an even number of heads per
 // group): the work is split into runs of blocks per head pair (runs.cuh); three launches:

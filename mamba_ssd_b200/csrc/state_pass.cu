@@ -16,6 +16,7 @@
 // eight chunks issued together so the chain costs one memory round trip per eight chunks.
 // The pass is HBM/L2 bound (it touches each chunk state twice).
 #include "common.cuh"
+#include "items.cuh"
 #include "launch.h"
 #include "tc.cuh"
 
@@ -67,12 +68,20 @@ __global__ void __launch_bounds__(256) state_pass_kernel(float *__restrict__ sta
 // per block, consecutive threads walking p then n, so every warp access is contiguous.  Four
 // blocks' loads per round trip and at most 48 registers, so five CTAs share an SM and the
 // whole grid (B*H*P*N/4 threads: 640 CTAs for the 2.7B shape) is resident in one wave.
+// The tensor-core workspace: block gb's decay factors of head h are the 128 floats at
+// (h * nblocks + gb) * 128 (head-major), its states at (gb * H + h) * P * N (block-major).  A packed varlen batch
+// (vl.n > 0) chains each sequence's own blocks, from the h0 of its index among the caller's
+// sequences to that sequence's h_final; grid.z walks the sequences.
+// VARLEN is a template parameter so that the equal-length instantiation carries none of the
+// table lookup (it fits its 48 registers without spilling).
+template <bool VARLEN>
 __global__ void __launch_bounds__(256, 5) state_pass_t_kernel(const float *__restrict__ statesT,
                                                            const float *__restrict__ acs2,
                                                            const float *__restrict__ h0,
                                                            float *__restrict__ h_final,
                                                            __nv_bfloat16 *__restrict__ hT, int H,
-                                                           int P, int N, int nc, int Q) {
+                                                           int P, int N, int nk, int Q, int nblocks,
+                                                           const Varlen vl) {
     constexpr int kAhead = 4;
     grid_dependency_wait();  // the block states come from the kernel before
     statesT = after_wait(statesT);
@@ -82,15 +91,28 @@ __global__ void __launch_bounds__(256, 5) state_pass_t_kernel(const float *__res
     hT = after_wait(hT);
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     const int p0 = (t * 4) % P, n = (t * 4) / P;
-    const int h = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.y;
     if (n >= N) return;
-    const size_t bh = (size_t)b * H + h;
+    // the sequence's first block, its block count, and where its h0 / h_final are
+    int gb0 = blockIdx.z * nk, nc = nk, seq = blockIdx.z;
+    if (VARLEN) {
+        const int *blk0 = after_wait(vl.blk0);
+        gb0 = blk0[blockIdx.z];
+        nc = blk0[blockIdx.z + 1] - gb0;
+        seq = after_wait(vl.seq)[blockIdx.z];
+    }
+    const size_t bh = (size_t)seq * H + h;
     const size_t PN = (size_t)P * N;
     float s[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) s[i] = h0 ? h0[bh * PN + (size_t)(p0 + i) * N + n] : 0.f;
-    const float *a_last = acs2 + bh * (size_t)nc * Q + (Q - 1);
-    const size_t off = (size_t)n * P + p0;
+    // running pointers to this thread's element of block gb0 + c; consecutive blocks of one head
+    // are H*P*N state elements apart (and 128 factor floats)
+    const size_t step = (size_t)H * PN;
+    const size_t first = ((size_t)gb0 * H + h) * PN + (size_t)n * P + p0;
+    const float *src = statesT + first;
+    __nv_bfloat16 *dst = hT + first;
+    const float *a_last = acs2 + ((size_t)h * nblocks + gb0) * Q + (Q - 1);
     // the block states' last read: marked first to leave L2, which keeps the h_prev^T just
     // written there for the scan
     const uint64_t release = tc::l2_evict_first();
@@ -100,9 +122,8 @@ __global__ void __launch_bounds__(256, 5) state_pass_t_kernel(const float *__res
 #pragma unroll
         for (int j = 0; j < kAhead; ++j) {
             if (c0 + j < nc) {
-                in[j] = ld_global_hint(reinterpret_cast<const float4 *>(statesT + (((size_t)b * nc + c0 + j) * H + h) * PN + off),
-                                       release);
-                a[j] = a_last[(size_t)(c0 + j) * Q];
+                in[j] = ld_global_hint(reinterpret_cast<const float4 *>(src + j * step), release);
+                a[j] = a_last[j * Q];
             }
         }
 #pragma unroll
@@ -111,7 +132,7 @@ __global__ void __launch_bounds__(256, 5) state_pass_t_kernel(const float *__res
                 __nv_bfloat162 lo2 = __floats2bfloat162_rn(s[0], s[1]);
                 __nv_bfloat162 hi2 = __floats2bfloat162_rn(s[2], s[3]);
                 uint2 v = make_uint2(*reinterpret_cast<uint32_t *>(&lo2), *reinterpret_cast<uint32_t *>(&hi2));
-                *reinterpret_cast<uint2 *>(hT + (((size_t)b * nc + c0 + j) * H + h) * PN + off) = v;
+                *reinterpret_cast<uint2 *>(dst + j * step) = v;
                 const float d = exp2f(a[j]);  // acs arrives as acs * log2(e) on this path
                 s[0] = fmaf(d, s[0], in[j].x);
                 s[1] = fmaf(d, s[1], in[j].y);
@@ -119,6 +140,9 @@ __global__ void __launch_bounds__(256, 5) state_pass_t_kernel(const float *__res
                 s[3] = fmaf(d, s[3], in[j].w);
             }
         }
+        src += kAhead * step;
+        dst += kAhead * step;
+        a_last += kAhead * Q;
     }
     if (h_final) {
 #pragma unroll
@@ -128,12 +152,15 @@ __global__ void __launch_bounds__(256, 5) state_pass_t_kernel(const float *__res
 }
 
 cudaError_t launch_state_pass_t(const float *states, const float *acs, const float *h0, float *h_final,
-                                __nv_bfloat16 *hT, int B, int L, int H, int P, int N, int chunk,
-                                cudaStream_t st) {
-    const int nc = cdiv(L, chunk);
-    dim3 grid(cdiv(P * N / 4, 256), H, B);
-    return launch_pdl(state_pass_t_kernel, grid, dim3(256), 0, st, states, acs, h0, h_final, hT, H, P, N, nc,
-                      chunk);
+                                __nv_bfloat16 *hT, int B, int L, int H, int P, int N, int chunk, const Varlen &vl,
+                                int nblocks, cudaStream_t st) {
+    const int nk = cdiv(L, chunk);
+    dim3 grid(cdiv(P * N / 4, 256), H, vl.n ? vl.n : B);
+    if (vl.n)
+        return launch_pdl(state_pass_t_kernel<true>, grid, dim3(256), 0, st, states, acs, h0, h_final, hT, H, P, N, nk,
+                          chunk, nblocks, vl);
+    return launch_pdl(state_pass_t_kernel<false>, grid, dim3(256), 0, st, states, acs, h0, h_final, hT, H, P, N, nk,
+                      chunk, nblocks, vl);
 }
 
 cudaError_t launch_state_pass(float *states, const float *acs, const float *h0, float *h_final,

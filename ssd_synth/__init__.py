@@ -223,3 +223,11 @@ def norm_inputs(T, C, dtype="bf16", seed=0):
     z = rng.standard_normal((T, C), dtype=np.float32)
     w = rng.uniform(0.5, 1.5, size=C).astype(np.float32)
     return {"y": to_storage(y, dtype), "z": to_storage(z, dtype), "w": _f32(w)}
+
+
+def varlen_lengths(n=64, lo=64, hi=4096, seed=2024):
+    """Lengths of a packed varlen batch: n sequences of lo .. hi tokens, log-uniform (many short
+    sequences beside a few long ones, as in a serving batch of prompts).  The default is the
+    batch the varlen bench leg times: 64 sequences, 51908 tokens, 439 blocks of 128."""
+    rng = np.random.default_rng(seed)
+    return [int(v) for v in np.exp(rng.uniform(np.log(lo), np.log(hi), n)).round()]

@@ -39,7 +39,7 @@ def test_status_strings_and_version():
     for s in range(6):
         assert L.ssd_status_string(s)
     assert L.ssd_status_string(99) == b"unknown status"
-    assert L.ssd_abi_version() == 4
+    assert L.ssd_abi_version() == 5
     assert L.ssd_last_cuda_error() == 0
 
 
@@ -220,13 +220,39 @@ def varlen(cu, **kw):
     (None, {}, INV), ([0, 5], dict(n=-1), INV), ([1, 5], {}, INV), ([0, 5, 3], {}, INV),
     ([0, 5], dict(x=None), INV), ([0, 5], dict(dt=MIS), INV), ([0, 5], dict(A_log=None), INV),
     ([0, 5], dict(P=32), UNS), ([0, 5], dict(chunk=100), UNS),
-    ([0, 1, 4], dict(H=4), UNS),          # bf16 dt rows of sequence 1 would start 8 bytes in
+    # the per-sequence (CUDA-core) path: f32 dt rows of sequence 1 would start 8 bytes in; the
+    # one-pass tensor-core path reads the packed tensors from their bases and takes any start
+    ([0, 1, 4], dict(H=2, N=16, dtype=F32), UNS),
     ([0, 5], dict(ws=None), WS), ([0, 5], dict(ws_bytes=256), WS), ([0, 5], dict(ws=A + 16), WS),
     ([0], {}, OK), ([0, 0, 0], dict(x=None, dt=None, Bm=None, Cm=None, y=None, n=0), OK),
 ])
 def test_varlen_validation(cu, kw, want):
     # every case is decided before a launch, so it runs without a GPU
     assert varlen(cu, **kw) == want
+
+
+def varlen_size(cu, H=80, P=64, G=1, N=128, chunk=256, dtype=BF16):
+    arr = (ctypes.c_int * len(cu))(*cu)
+    return L.ssd_chunk_scan_varlen_workspace_size(ctypes.cast(arr, ctypes.c_void_p), len(cu) - 1, H, P, G, N, chunk,
+                                                  dtype)
+
+
+def test_varlen_workspace_size():
+    # one pass (bf16, P = 64, N = 128): the block-major prefill workspace of every block of the
+    # batch, then the table (three int arrays of m + 1 entries, m non-empty sequences, each in
+    # a 256-byte slot)
+    cu = [0, 100, 100, 400, 4496]  # blocks 1 + 0 + 3 + 32 = 36, three non-empty sequences
+    nb, H, P, N = 36, 80, 64, 128
+    prefill = 256 + 2 * (4 * H * nb * 128) + 4 * nb * H * P * N + 2 * nb * H * P * N
+    assert varlen_size(cu) == prefill + 3 * 256
+    assert varlen_size(cu) == L.ssd_chunk_scan_workspace_size(1, nb * 128, H, P, 1, N, 256, BF16) + 3 * 256
+    # the per-sequence path: the longest sequence's prefill workspace, shared
+    assert varlen_size(cu, dtype=F32) == L.ssd_chunk_scan_workspace_size(1, 4096, H, P, 1, N, 256, F32)
+    assert varlen_size([0]) == 0
+    assert varlen_size([0, 5, 3]) == 0    # decreasing
+    assert varlen_size([2, 5]) == 0       # not starting at 0
+    assert varlen_size([0, 5], P=32) == 0
+    assert varlen_size([0, 0, 0]) == 256 + 3 * 256  # no blocks: the status slot and the table
 
 
 def test_header_is_plain_c_and_links(tmp_path):
