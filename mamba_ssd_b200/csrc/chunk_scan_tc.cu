@@ -83,8 +83,8 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_h,
     const __grid_constant__ CUtensorMap tm_y, const float *__restrict__ dtf, const float *__restrict__ acs,
-    const float *__restrict__ D, __nv_bfloat16 *__restrict__ y, int *__restrict__ status, int L, int H, int G,
-    int nk, int total, const Varlen vl) {
+    const float *__restrict__ D, __nv_bfloat16 *__restrict__ y, const __nv_bfloat16 *__restrict__ hT,
+    int *__restrict__ status, int L, int H, int G, int nk, int total, const Varlen vl) {
     using namespace csc;
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
@@ -143,6 +143,7 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
     acs = after_wait(acs);
     D = after_wait(D);
     y = after_wait(y);
+    hT = after_wait(hT);
     status = after_wait(status);
     const Varlen tab = {after_wait(vl.tok0), after_wait(vl.blk0), after_wait(vl.seq), vl.n};
 
@@ -372,6 +373,10 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[t]);
+                // the item's h_prev^T tile (128 rows of 128 bytes) was read by its TMA load, which
+                // completed before the MMA that produced O: it is dead, and its lines leave L2
+                // without a write-back (only this item reads them)
+                if (half == 0) discard_l2_line(hT + ((size_t)it.gblk() * H + h) * N * P + (size_t)myrow * P);
                 const float scale = ex2_approx(al);
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
@@ -445,7 +450,7 @@ cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, 
         cudaError_t r = raise_smem_limit<kernel>((int)kSmem);
         if (r != cudaSuccess) return r;
         return launch_pdl(kernel, dim3(grid), dim3(kThreads), kSmem, st, tm_x, tm_b, tm_c, tm_h, tm_y, dtf, acs, D,
-                          (__nv_bfloat16 *)y, status, L, H, G, nk, total, vl);
+                          (__nv_bfloat16 *)y, hT, status, L, H, G, nk, total, vl);
     };
     return vl.n ? launch(KernelTag<chunk_scan_tc_kernel<true>>{}) : launch(KernelTag<chunk_scan_tc_kernel<false>>{});
 }

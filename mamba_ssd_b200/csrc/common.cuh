@@ -83,6 +83,14 @@ __device__ __forceinline__ T *after_wait(T *p) {
     return p;
 }
 
+// Drop the 128-byte L2 line at p (128-byte aligned) without writing it back: for a workspace
+// intermediate whose last read has happened (by every thread that reads it, in a happens-before
+// order), so that its dirty line never costs a DRAM write.  The line's contents become
+// undefined.
+__device__ __forceinline__ void discard_l2_line(const void *p) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
 // A global load with an L2 eviction-priority policy (a createpolicy result).
 __device__ __forceinline__ float4 ld_global_hint(const float4 *p, uint64_t policy) {
     float4 v;

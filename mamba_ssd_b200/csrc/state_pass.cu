@@ -92,6 +92,8 @@ __global__ void __launch_bounds__(256, 5) state_pass_t_kernel(const float *__res
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     const int p0 = (t * 4) % P, n = (t * 4) / P;
     const int h = blockIdx.y;
+    // (n < N for every thread of the tensor-core shape, P * N / 4 being a multiple of 256: no
+    // warp is split by this exit, which the warp-wide steps below rely on)
     if (n >= N) return;
     // the sequence's first block, its block count, and where its h0 / h_final are
     int gb0 = blockIdx.z * nk, nc = nk, seq = blockIdx.z;
@@ -139,6 +141,15 @@ __global__ void __launch_bounds__(256, 5) state_pass_t_kernel(const float *__res
                 s[2] = fmaf(d, s[2], in[j].z);
                 s[3] = fmaf(d, s[3], in[j].w);
             }
+        }
+        // the block states just read are dead (only this pass reads them): their lines leave L2
+        // without a write-back.  Every lane's loads have returned (their values are used
+        // above); lanes 0, 8, 16, 24 each own one 128-byte line of the warp's 512 bytes.
+        __syncwarp();
+        if ((threadIdx.x & 7) == 0) {
+#pragma unroll
+            for (int j = 0; j < kAhead; ++j)
+                if (c0 + j < nc) discard_l2_line(src + j * step);
         }
         src += kAhead * step;
         dst += kAhead * step;

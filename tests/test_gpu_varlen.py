@@ -7,6 +7,8 @@ sequences (more than one table launch carries), the 64-sequence 2.7B-shaped batc
 times (checked on sampled heads), sequences starting at odd tokens, and the call captured in
 a CUDA graph and replayed on new contents.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -97,6 +99,8 @@ def test_varlen_bench_batch_sampled_heads():
     check_close(host64(hf)[:, heads], h_ref, "bf16", "h", "bench batch h_final, sampled heads")
 
 
+@pytest.mark.skipif(os.environ.get("SSD_PREFILL_KERNELS") in ("simt", "fused"),
+                    reason="the per-sequence path these switches select rejects unaligned starts (tested below)")
 def test_varlen_odd_starts_one_pass():
     # H = 4 bf16: dt rows are 8 bytes, so sequences start off 16-byte boundaries; the one-pass
     # path reads the packed tensors from their bases and takes any start
