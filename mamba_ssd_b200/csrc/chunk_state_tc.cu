@@ -331,6 +331,9 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
         const int quarter = warp & 3, half = (warp - 2 - kXform) >> 2;
         const int n = quarter * 32 + lane;
         const bool leader = warp == 2 + kXform && lane == 0;  // issues the stores
+        // the block states stay in L2 for the state pass, which reads them next and then drops
+        // their lines (they are never needed in DRAM)
+        const uint64_t keep = l2_evict_last();
         uint8_t *box = smem + kOffOut + half * kBox;
         ItemCursor<VARLEN> it(first, H, G, nk, L, tab);
         for (int j = 0; j < cnt; ++j, it.next()) {
@@ -364,8 +367,8 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
             named_barrier(kEpiBar, kEpi * 32);
             if (leader) {
                 const int row = (int)(((size_t)it.gblk() * H + it.h()) * N);
-                tma_store_2d(&tm_s, smem + kOffOut, 0, row);
-                tma_store_2d(&tm_s, smem + kOffOut + kBox, 32, row);
+                tma_store_2d_hint(&tm_s, smem + kOffOut, 0, row, keep);
+                tma_store_2d_hint(&tm_s, smem + kOffOut + kBox, 32, row, keep);
                 bulk_commit();
             }
         }

@@ -115,10 +115,16 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, int
         : "memory");
 }
 
-// L2 eviction-priority policy for the cache-hinted loads below.  A tensor's last read within a
-// prefill call (x, the block states, h_prev^T) is marked evict_first, so that it leaves L2 ahead
-// of data a later kernel of the call still reads: the block states the state pass reads right
-// after chunk_state_tc writes them, and the h_prev^T the scan reads after the state pass.
+// L2 eviction-priority policies for the cache-hinted copies below.  A tensor's last read within
+// a prefill call (x, the block states, h_prev^T) is marked evict_first, so that it leaves L2
+// ahead of data a later kernel of the call still reads: the block states the state pass reads
+// right after chunk_state_tc writes them (stored evict_last), and the h_prev^T the scan reads
+// after the state pass.
+__device__ __forceinline__ uint64_t l2_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
 __device__ __forceinline__ uint64_t l2_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -164,6 +170,13 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *s
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
                      reinterpret_cast<uint64_t>(m)),
                  "r"(smem_u32(src)), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap *m, const void *src, int c0, int c1,
+                                                  uint64_t policy) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1), "l"(policy)
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
