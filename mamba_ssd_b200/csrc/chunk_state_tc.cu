@@ -66,7 +66,7 @@ constexpr uint32_t kStageBytes = 2 * kBox + 1024;  // x/hi box, lo box, ldt[128]
 constexpr uint32_t kOffStage = 2 * kBox;
 constexpr uint32_t kOffOut = kOffStage + kStages * kStageBytes;  // S^T staging: 2 x [128][32] fp32
 constexpr uint32_t kOffBar = kOffOut + 2 * kBox;
-constexpr int kEpiBar = 1;  // named barrier of the epilogue warps
+constexpr int kEpiBar = 1;  // named barriers of the epilogue's two column halves: 1 and 2
 constexpr uint32_t kSmem = kOffBar + 256 + 1024;  // + slack for 1024-byte alignment
 constexpr uint32_t kTmemCols = 256;               // two 128-column fp32 accumulators [hi | lo]
 }  // namespace cst
@@ -328,9 +328,13 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
     } else {
         // ---------------------------------------------------------------- epilogue
         // TMEM lane quarter (warp % 4) = rows n, column half = p range of 32
+        // The two column halves (4 warps each, one TMEM lane quarter per warp) drain, stage and
+        // store their own 32-column box independently: each half has its own named barrier and
+        // its own TMA store, so neither waits for the other.
         const int quarter = warp & 3, half = (warp - 2 - kXform) >> 2;
         const int n = quarter * 32 + lane;
-        const bool leader = warp == 2 + kXform && lane == 0;  // issues the stores
+        const bool leader = ((warp - 2 - kXform) & 3) == 0 && lane == 0;  // issues this half's stores
+        const int bar = kEpiBar + half;
         // the block states stay in L2 for the state pass, which reads them next and then drops
         // their lines (they are never needed in DRAM)
         const uint64_t keep = l2_evict_last();
@@ -358,17 +362,16 @@ __global__ void __launch_bounds__(cst::kThreads, 1) chunk_state_tc_kernel(
             }
             // the staging tile is free once the previous item's stores have read it
             if (leader) bulk_wait_read();
-            if (!named_barrier_and(kEpiBar, kEpi * 32, ok)) break;
+            if (!named_barrier_and(bar, kEpi / 2 * 32, ok)) break;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
                 *reinterpret_cast<float4 *>(box + sw128_offset(n, c)) =
                     make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
             fence_proxy_async_smem();
-            named_barrier(kEpiBar, kEpi * 32);
+            named_barrier(bar, kEpi / 2 * 32);
             if (leader) {
                 const int row = (int)(((size_t)it.gblk() * H + it.h()) * N);
-                tma_store_2d_hint(&tm_s, smem + kOffOut, 0, row, keep);
-                tma_store_2d_hint(&tm_s, smem + kOffOut + kBox, 32, row, keep);
+                tma_store_2d_hint(&tm_s, box, half * 32, row, keep);
                 bulk_commit();
             }
         }
