@@ -40,8 +40,9 @@
 //                the item's per-token factors into a ring of kStages stages
 //   warp 1       MMA issuer (one lane): CB per tile; O and Y per item into one of two TMEM sets
 //   warps 2..9   P~ of an item into its TMEM set
-//   warps 10..17 epilogue: y = Y + exp(acs) O of an item into a swizzled shared-memory tile
-//                that one TMA store writes out (tokens past L are clipped by the store); the
+//   warps 10..17 epilogue: y = Y + exp(acs) O of an item; each 32-column half (4 warps) stages
+//                its columns in its own swizzled shared-memory box that its own TMA store
+//                writes out (tokens past L are clipped by the store); the
 //                ragged last block of a packed varlen sequence is stored row by row instead,
 //                its real rows only, since the rows after it belong to the next sequence
 //                (their P~ rows only ever meet x rows after the sequence's end through the
@@ -75,7 +76,7 @@ constexpr uint32_t kSmem = kOffBar + 256 + 1024;
 constexpr uint32_t kColCB = 0, kSet = 192, kSet0 = 128, kOffPT = 0, kOffY = 64, kOffO = 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kDiagFactorRange = 96.f;  // log2 range of a diagonal sub-block that is factored
-constexpr int kEpiBar = 1;                 // named barrier of the epilogue warps
+constexpr int kEpiBar = 1;                 // named barriers of the epilogue's two column halves: 1, 2
 }  // namespace csc
 
 template <bool VARLEN>
@@ -350,7 +351,12 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
         const int rq = warp & 3, half = (warp - 2 - kPt) >> 2;  // TMEM lane quarter, 32 columns
         const int myrow = rq * 32 + lane;
         const uint32_t lane_base = (uint32_t)(rq * 32) << 16;
-        const bool leader = warp == 2 + kPt && lane == 0;  // issues the stores
+        // The two column halves (4 warps each, one TMEM lane quarter per warp) stage and store
+        // their own 32-column box (64-byte rows, 64-byte swizzle) with their own named barrier
+        // and TMA store, so neither waits for the other.
+        const bool leader = ((warp - 2 - kPt) & 3) == 0 && lane == 0;  // issues this half's stores
+        const int bar = kEpiBar + half;
+        uint8_t *box = smem + kOffOut + half * (kBox / 2);
         ItemCursor<VARLEN> it(first, H, G, nk, L, tab);
         for (int j = 0; j < cnt; ++j, it.next()) {
             const int t = j & 1, h = it.h();
@@ -384,7 +390,7 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
             }
             // the staging tile is free once the previous item's store has read it
             if (leader) bulk_wait_read();
-            if (!named_barrier_and(kEpiBar, kEpi * 32, ok)) break;
+            if (!named_barrier_and(bar, kEpi / 2 * 32, ok)) break;
             if (direct < R) {  // item-uniform
                 if (myrow < direct) {
                     uint4 *dst = reinterpret_cast<uint4 *>(y + ((size_t)it.row() + myrow) * H * P + (size_t)h * P +
@@ -396,12 +402,12 @@ __global__ void __launch_bounds__(csc::kThreads, 1) chunk_scan_tc_kernel(
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4 *>(smem + kOffOut + sw128_offset(myrow, half * 4 + q)) =
+                *reinterpret_cast<uint4 *>(box + sw64_offset(myrow, q)) =
                     make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
             fence_proxy_async_smem();
-            named_barrier(kEpiBar, kEpi * 32);
+            named_barrier(bar, kEpi / 2 * 32);
             if (leader) {
-                tma_store_3d(&tm_y, smem + kOffOut, h * P, it.row(), it.zb);
+                tma_store_3d(&tm_y, box, h * P + half * 32, it.row(), it.zb);
                 bulk_commit();
             }
         }
@@ -441,8 +447,9 @@ cudaError_t launch_chunk_scan_tc(const void *x, const void *Bm, const void *Cm, 
     if (e != cudaSuccess) return e;
     e = make_tmap_bf16_2d(&tm_h, hT, (uint64_t)P, (uint64_t)nblocks * H * N, (uint64_t)P * 2, 64, R);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16_3d(&tm_y, y, (uint64_t)H * P, (uint64_t)L, (uint64_t)B, (uint64_t)H * P * 2,
-                          (uint64_t)L * H * P * 2, 64, R, 1);
+    // y leaves in 32-column boxes, one per epilogue half
+    e = make_tmap_bf16_3d_sw64(&tm_y, y, (uint64_t)H * P, (uint64_t)L, (uint64_t)B, (uint64_t)H * P * 2,
+                               (uint64_t)L * H * P * 2, 32, R, 1);
     if (e != cudaSuccess) return e;
     const int grid = total < num_sms ? total : num_sms;
     auto launch = [&](auto tag) {

@@ -41,8 +41,9 @@
 //                serves the items of stage s)
 //   warp 1       MMA issuer (one lane): 8 MMAs per item into one of two TMEM accumulators
 //   warps 2..9   transform: scale rows by w into hi (in place) and lo
-//   warps 10..17 epilogue: drain an accumulator through a swizzled shared-memory tile that
-//                one TMA store per 32-column half writes out (S^T, [N][P], fp32)
+//   warps 10..17 epilogue: drain an accumulator; each 32-column half (4 warps) stages its
+//                columns in its own swizzled shared-memory box and writes them out with its own
+//                TMA store (S^T, [N][P], fp32)
 // Every role runs its own loop and the roles meet only at mbarriers (full/empty per stage,
 // per accumulator, per B tile), so the tensor core, the transform of the next item and the
 // drain of the previous one overlap.

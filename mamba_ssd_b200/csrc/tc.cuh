@@ -300,6 +300,11 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
 __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
     return (uint32_t)row * 128u + (uint32_t)((chunk ^ (row & 7)) << 4);
 }
+// The same for a box of 64-byte rows under 64-byte swizzle (the 16-byte chunk index, 0..3,
+// XORed with bits 7..8 of the row's byte offset).
+__device__ __forceinline__ uint32_t sw64_offset(int row, int chunk) {
+    return (uint32_t)row * 64u + (uint32_t)((chunk ^ ((row >> 1) & 3)) << 4);
+}
 
 // 2^x by the hardware approximation (relative error ~2^-22, flushes results below the fp32
 // normal range to 0).

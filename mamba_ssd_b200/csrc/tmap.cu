@@ -26,6 +26,30 @@ void resolve() {
 }
 }  // namespace
 
+namespace {
+cudaError_t bf16_3d(CUtensorMap *out, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                    uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1, uint32_t box2,
+                    CUtensorMapSwizzle swizzle) {
+    std::call_once(g_once, resolve);
+    if (!g_encode) return cudaErrorNotSupported;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+    cuuint32_t box[3] = {box0, box1, box2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+}  // namespace
+
+cudaError_t make_tmap_bf16_3d_sw64(CUtensorMap *out, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
+                                   uint32_t box2) {
+    return bf16_3d(out, base, d0, d1, d2, stride1_bytes, stride2_bytes, box0, box1, box2,
+                   CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 cudaError_t make_tmap_bf16_3d(CUtensorMap *out, const void *base, uint64_t d0, uint64_t d1,
                               uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes,
                               uint32_t box0, uint32_t box1, uint32_t box2) {

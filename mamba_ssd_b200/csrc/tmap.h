@@ -14,6 +14,11 @@ cudaError_t make_tmap_bf16_3d(CUtensorMap *out, const void *base, uint64_t d0, u
                               uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes,
                               uint32_t box0, uint32_t box1, uint32_t box2);
 
+// The same with 64-byte swizzle (box0 * 2 bytes must be <= 64).
+cudaError_t make_tmap_bf16_3d_sw64(CUtensorMap *out, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
+                                   uint32_t box2);
+
 // A 2-D bf16 tensor map with 128-byte swizzle: dims d0 (inner), d1; byte stride of dim 1.
 cudaError_t make_tmap_bf16_2d(CUtensorMap *out, const void *base, uint64_t d0, uint64_t d1,
                               uint64_t stride1_bytes, uint32_t box0, uint32_t box1);
