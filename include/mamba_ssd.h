@@ -119,7 +119,11 @@ SSD_API size_t ssd_chunk_scan_workspace_size(int B, int L, int H, int P, int G, 
  *   chunk                              tokens per chunk; the last chunk may be ragged
  *   workspace, workspace_bytes         >= ssd_chunk_scan_workspace_size(...), 256-byte
  *                                      aligned, contents on entry irrelevant; it is
- *                                      scratch for this call only
+ *                                      scratch for this call only, and after the call
+ *                                      only its status word (ssd_chunk_scan_status) is
+ *                                      defined: the tensor-core kernels drop the block
+ *                                      states and h_prev from L2 once read, without
+ *                                      writing them back
  * Supported: H % G == 0, P == 64, N in {16, 32, 64, 128}, chunk in {64, 128, 256, 512},
  * L >= 0, B >= 0.  Other valid shapes return SSD_ERR_UNSUPPORTED.  Calls sharing a
  * workspace must be ordered on one stream.
