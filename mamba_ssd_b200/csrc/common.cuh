@@ -91,6 +91,20 @@ __device__ __forceinline__ void discard_l2_line(const void *p) {
     asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
 }
 
+// 16-byte L2-only load / global store with an L2 eviction-priority policy (a createpolicy result).
+__device__ __forceinline__ float4 ldcg_hint(const float4 *p, uint64_t policy) {
+    float4 v;
+    asm volatile("ld.global.cg.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p), "l"(policy));
+    return v;
+}
+__device__ __forceinline__ void st_global_hint_v4(float4 *p, float4 v, uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w), "l"(policy)
+                 : "memory");
+}
+
 // A global load with an L2 eviction-priority policy (a createpolicy result).
 __device__ __forceinline__ float4 ld_global_hint(const float4 *p, uint64_t policy) {
     float4 v;

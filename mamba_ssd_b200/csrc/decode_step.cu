@@ -33,6 +33,7 @@
 // waits; kernel 2 resets the workspace status word to SSD_OK and never sets it otherwise.
 #include "common.cuh"
 #include "launch.h"
+#include "tc.cuh"
 
 namespace ssd {
 
@@ -88,7 +89,8 @@ __global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(
 template <typename T, int N, int ROWS, int THREADS>
 __global__ void __launch_bounds__(THREADS) decode_state_kernel(
     float *__restrict__ ssm, const float *__restrict__ u_ws, const float2 *__restrict__ da_ws,
-    const float *__restrict__ D, T *__restrict__ y_t, int H, int P, int G, int *__restrict__ status) {
+    const float *__restrict__ D, T *__restrict__ y_t, int H, int P, int G, int *__restrict__ status,
+    int stream_first) {
     constexpr int V = (N > 128) ? N / 128 : 1;  // float4 per thread per row
     constexpr int TPR = N / (4 * V);            // threads per row (<= 32, power of two)
     constexpr int RPP = THREADS / TPR;          // rows per pass
@@ -104,6 +106,10 @@ __global__ void __launch_bounds__(THREADS) decode_state_kernel(
     const int r_in_pass = threadIdx.x / TPR, lane_in_row = threadIdx.x % TPR;
 
     // ---- the state, before the dependency wait: L2-only loads (see the file comment) ----
+    // With stream_first the state's lines are loaded and stored evict_first: at small batches
+    // that keeps the step's small data (the conv windows and taps, the conv outputs) in L2
+    // across the 64-layer stream of states.
+    const uint64_t first_policy = tc::l2_evict_first();
     float4 st[PASSES][V];
     float *ssm_b = ssm + ((size_t)b * HP + row0) * N;
 #pragma unroll
@@ -112,8 +118,10 @@ __global__ void __launch_bounds__(THREADS) decode_state_kernel(
 #pragma unroll
         for (int v = 0; v < V; ++v)
             if (r < ROWS)
-                st[ps][v] = __ldcg(reinterpret_cast<const float4 *>(ssm_b + (size_t)r * N +
-                                                                    (v * TPR + lane_in_row) * 4));
+            {
+                const float4 *src = reinterpret_cast<const float4 *>(ssm_b + (size_t)r * N + (v * TPR + lane_in_row) * 4);
+                st[ps][v] = stream_first ? ldcg_hint(src, first_policy) : __ldcg(src);
+            }
     }
 
     grid_dependency_wait();  // the conv kernel's u and (dt, a) are complete and visible
@@ -162,7 +170,11 @@ __global__ void __launch_bounds__(THREADS) decode_state_kernel(
                 part = fmaf(s.y, uC[v].y, part);
                 part = fmaf(s.z, uC[v].z, part);
                 part = fmaf(s.w, uC[v].w, part);
-                *reinterpret_cast<float4 *>(ssm_b + (size_t)r * N + (v * TPR + lane_in_row) * 4) = s;
+                float4 *dst = reinterpret_cast<float4 *>(ssm_b + (size_t)r * N + (v * TPR + lane_in_row) * 4);
+                if (stream_first)
+                    st_global_hint_v4(dst, s, first_policy);
+                else
+                    *dst = s;
             }
         }
 #pragma unroll
@@ -202,6 +214,11 @@ cudaError_t launch_decode_conv(int dtype, void *conv_state, const void *xBC_t, c
                          da_ws, B, H, Cc, st);
 }
 
+// Batches up to this size stream the state evict_first.  Measured on the 64-layer 2.7B-shaped
+// decode (steps/s, against the default policy): +14 % at batch 1, +5 % at 2, +1 % at 4, -3 % at
+// 8 and 16.
+constexpr int kStreamFirstMaxB = 4;
+
 template <typename T, int N>
 static cudaError_t state_launch(float *ssm, const float *u_ws, const float2 *da_ws, const float *D, void *y_t,
                                 int B, int H, int P, int G, int *status, cudaStream_t st) {
@@ -210,7 +227,7 @@ static cudaError_t state_launch(float *ssm, const float *u_ws, const float2 *da_
     constexpr int THREADS = ROWS * TPR < 128 ? ROWS * TPR : 128;
     const dim3 grid(H * P / ROWS, B);
     return launch_pdl(decode_state_kernel<T, N, ROWS, THREADS>, grid, dim3(THREADS), 0, st, ssm, u_ws, da_ws,
-                      D, (T *)y_t, H, P, G, status);
+                      D, (T *)y_t, H, P, G, status, B <= kStreamFirstMaxB ? 1 : 0);
 }
 
 cudaError_t launch_decode_state(int dtype, float *ssm_state, const float *u_ws, const float2 *da_ws,
