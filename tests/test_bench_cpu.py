@@ -1,6 +1,6 @@
 """Host-side arithmetic of bench.py (CPU only): the algorithmic bytes per unit that the
 roofline divides by, the gate that reports ncu traffic only for unchanged kernel sources,
-and the decode-vs-recompute ratio."""
+the decode-vs-recompute ratio, and the varlen leg's batch."""
 import json
 import os
 import sys
@@ -61,3 +61,16 @@ def test_decode_vs_recompute_ratio():
     assert r["speedup"] == pytest.approx(20.0)
     assert r["context"] == bench.PF["L"] and r["by_context"] == [{"L": 1024}]
     assert bench.decode_vs_recompute(5.0, {}) is None
+
+
+def test_varlen_bench_batch():
+    # the packed batch the varlen leg times (and the GPU test checks on sampled heads): 64
+    # sequences of 64 .. 4096 tokens, log-uniform, seeded, the same on every call
+    import ssd_synth as S
+    lengths = S.varlen_lengths()
+    assert lengths == S.varlen_lengths()
+    assert len(lengths) == 64 and min(lengths) >= 64 and max(lengths) <= 4096
+    assert sum(lengths) == 51908
+    assert sum(-(-n // 128) for n in lengths) == 439  # 128-token blocks of the one-pass kernels
+    # a wide spread: a few long sequences beside many short ones
+    assert sum(n >= 2048 for n in lengths) < sum(n < 512 for n in lengths)
