@@ -39,6 +39,29 @@ namespace ssd {
 
 constexpr int kConvThreads = 256;
 
+// Loads and stores of one bf16 or fp32 element with an L2 eviction-priority policy: the conv
+// kernel keeps the conv windows and taps evict_last, so that the 64-layer stream of states
+// between two steps of a layer does not push them out of L2.
+template <typename T> __device__ __forceinline__ T ld_policy(const T *p, uint64_t pol);
+template <> __device__ __forceinline__ __nv_bfloat16 ld_policy(const __nv_bfloat16 *p, uint64_t pol) {
+    unsigned short v;
+    asm volatile("ld.global.L2::cache_hint.b16 %0, [%1], %2;" : "=h"(v) : "l"(p), "l"(pol));
+    return __ushort_as_bfloat16(v);
+}
+template <> __device__ __forceinline__ float ld_policy(const float *p, uint64_t pol) {
+    float v;
+    asm volatile("ld.global.L2::cache_hint.f32 %0, [%1], %2;" : "=f"(v) : "l"(p), "l"(pol));
+    return v;
+}
+template <typename T> __device__ __forceinline__ void st_policy(T *p, T v, uint64_t pol);
+template <> __device__ __forceinline__ void st_policy(__nv_bfloat16 *p, __nv_bfloat16 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.b16 [%0], %1, %2;" ::"l"(p), "h"(__bfloat16_as_ushort(v)), "l"(pol)
+                 : "memory");
+}
+template <> __device__ __forceinline__ void st_policy(float *p, float v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
+}
+
 template <typename T, int K>
 __global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(
     T *__restrict__ conv_state, const T *__restrict__ xBC_t, const T *__restrict__ dt_t,
@@ -59,20 +82,21 @@ __global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(
     const int b = blockIdx.y;
     const int c = blockIdx.x * kConvThreads + threadIdx.x;
     if (c < Cc) {
+        const uint64_t keep = tc::l2_evict_last();
         T *cs = conv_state + ((size_t)b * Cc + c) * (K - 1);
         T win[K];
         float w[K];
 #pragma unroll
-        for (int k = 0; k < K - 1; ++k) win[k] = cs[k];
+        for (int k = 0; k < K - 1; ++k) win[k] = ld_policy(cs + k, keep);
         win[K - 1] = __ldg(xBC_t + (size_t)b * Cc + c);
 #pragma unroll
-        for (int k = 0; k < K; ++k) w[k] = to_f(__ldg(conv_w + (size_t)c * K + k));
-        float acc = conv_b ? to_f(__ldg(conv_b + c)) : 0.f;
+        for (int k = 0; k < K; ++k) w[k] = to_f(ld_policy(conv_w + (size_t)c * K + k, keep));
+        float acc = conv_b ? to_f(ld_policy(conv_b + c, keep)) : 0.f;
 #pragma unroll
         for (int k = 0; k < K; ++k) acc = fmaf(w[k], to_f(win[k]), acc);
         u_ws[(size_t)b * Cc + c] = silu_f(acc);
 #pragma unroll
-        for (int k = 0; k < K - 1; ++k) cs[k] = win[k + 1];
+        for (int k = 0; k < K - 1; ++k) st_policy(cs + k, win[k + 1], keep);
     }
     if (blockIdx.x == 0)
         for (int h = threadIdx.x; h < H; h += kConvThreads) {
