@@ -9,13 +9,26 @@
 // into their neighbours); the gate and the per-group RMS are the Mamba-2 block's norm, which
 // the pages name but do not spell out.
 //
-// One CTA per (token, norm group).  The group's GS channels stream in once as 16-byte vectors
-// of y and z; each thread keeps its gated values in shared memory (fp32) and adds up their
-// squares in fp32; the CTA reduces the sum, and a second pass over shared memory scales by the
-// reciprocal RMS and by w and streams the result out.  HBM-bound: 3 * GS * sizeof(T) bytes per
-// row (plus w, which stays in L2).  No waits of any kind.
+// HBM-bound: 3 * GS * sizeof(T) bytes per (token, group) row, plus w, which stays in L2.  Two
+// forms, neither with a spin-wait of any kind:
+//
+// Streaming form (a group's y row at most 20 KB: up to 10240 bf16 or 5120 float32 channels).
+// Persistent CTAs, as many as fit on the GPU at once, each walking rows gridDim.x apart.  A
+// thread owns 16 elements of a row (GS / 16 threads, rounded up to a warp).  While it works
+// on row k it has already asked for its 16-byte vectors of y and z of row k + 1: cp.async
+// copies them into the other half of a two-stage shared-memory ring.  Each thread reads back
+// only the vectors it copied itself, so waiting on its own copies (cp.async.wait_group) is
+// all the ordering the data needs; the one CTA barrier per row is the sum of squares.  A CTA
+// therefore always has a row of loads in flight, also while it reduces and stores.
+//
+// Staged form (larger groups, up to 32768 channels).  One CTA per (token, norm group).  The
+// group's GS channels stream in once as 16-byte vectors of y and z; each thread keeps its gated
+// values in shared memory (fp32) and adds up their squares in fp32; the CTA reduces the sum,
+// and a second pass over shared memory scales by the reciprocal RMS and by w and streams the
+// result out.
 #include "common.cuh"
 #include "launch.h"
+#include "tc.cuh"
 
 namespace ssd {
 
@@ -118,6 +131,173 @@ __global__ void __launch_bounds__(kNormThreads) gated_rmsnorm_kernel(const T *__
     allow_dependents();
 }
 
+constexpr int kNormStreamElems = 16;          // elements of a row per thread
+constexpr int kNormStreamRowBytes = 20480;    // largest y (or z) row of one group
+constexpr int kNormStreamMaxThreads = kNormStreamRowBytes / 2 / kNormStreamElems;  // bf16: 640
+
+__device__ __forceinline__ void cp_async16_first(void *smem, const void *gmem, uint64_t policy) {
+    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "l"(policy)
+                 : "memory");
+}
+// SiLU(z) = z / (1 + e^-z), with e^-z taken as 2^(-z log2 e) by the PTX approximate base-2
+// exponential and the division as a product with the approximate reciprocal, both in their
+// flush-to-zero forms (the build keeps denormals, and the non-flushing forms of those
+// instructions cost extra fix-up instructions per element).  Relative error about 2^-21;
+// a denormal z counts as zero.  -z is capped at 80 so that 1 + e^-z stays finite.
+__device__ __forceinline__ float silu_ftz(float z) {
+    float e, r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(fminf(-z, 80.f) * 1.4426950408889634f));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.f + e));
+    return z * r;
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_prior() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// rows: T_rows * n_groups (token-major, group fastest).  blockDim.x * VPT * VEC >= GS.
+template <typename T>
+__global__ void __launch_bounds__(kNormStreamMaxThreads) gated_rmsnorm_stream_kernel(
+    const T *__restrict__ y, const T *__restrict__ z, const float *__restrict__ w, T *__restrict__ out, int C,
+    int GS, int n_groups, int rows, float eps) {
+    constexpr int VEC = Vec16<T>::n;
+    constexpr int VPT = kNormStreamElems / VEC;  // 16-byte vectors of y (and of z) per thread
+    extern __shared__ __align__(16) uint4 ring_s[];  // [2 stages][y, z][GS / VEC vectors]
+    __shared__ __align__(16) float red[2][kNormStreamMaxThreads / 32];  // zero past the last warp
+
+    const int nthr = blockDim.x;
+    const int nwarp4 = ((nthr >> 5) + 3) & ~3;  // warps rounded up to a float4 of red
+    if (threadIdx.x < 2 * nwarp4) red[threadIdx.x / nwarp4][threadIdx.x % nwarp4] = 0.f;
+
+    grid_dependency_wait();  // y comes from the kernel before
+    y = after_wait(y);
+    z = after_wait(z);
+    w = after_wait(w);
+    out = after_wait(out);
+
+    const int nvec = GS / VEC;
+    const uint64_t first = tc::l2_evict_first();  // y and z are read once
+
+    // Rows r = t * n_groups + gi advance by gridDim.x = dt * n_groups + dg, so (t, gi) step by
+    // additions instead of divisions.
+    const int dt = gridDim.x / n_groups, dg = gridDim.x - dt * n_groups;
+    auto step = [&](int &t, int &gi) {
+        t += dt;
+        gi += dg;
+        if (gi >= n_groups) {
+            gi -= n_groups;
+            ++t;
+        }
+    };
+
+    // this thread's vectors of row (t, gi) into stage s; always one commit group per call
+    auto request = [&](int r, int t, int gi, int s) {
+        if (r < rows) {
+            const size_t base = (size_t)t * C + (size_t)gi * GS;
+            const uint4 *y4 = reinterpret_cast<const uint4 *>(y + base);
+            const uint4 *z4 = reinterpret_cast<const uint4 *>(z + base);
+            uint4 *sy = ring_s + (size_t)s * 2 * nvec;
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int v = threadIdx.x + i * nthr;
+                if (v < nvec) {
+                    cp_async16_first(sy + v, y4 + v, first);
+                    cp_async16_first(sy + nvec + v, z4 + v, first);
+                }
+            }
+        }
+        cp_async_commit();
+    };
+
+    int r = blockIdx.x;
+    int t = r / n_groups, gi = r - t * n_groups;  // row r's token and group
+    int tn = t, gn = gi;                          // those of row r + gridDim.x
+    step(tn, gn);
+    __syncthreads();  // red's zero padding
+    request(r, t, gi, 0);
+    for (int k = 0; r < rows; ++k, r += gridDim.x) {
+        request(r + gridDim.x, tn, gn, (k + 1) & 1);
+        cp_async_wait_prior();  // every group but the newest: row r's copies have landed
+
+        // ---- gate and sum of squares (fp32), from the vectors this thread copied ----
+        const uint4 *sy = ring_s + (size_t)(k & 1) * 2 * nvec;
+        float g[VPT][VEC];
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int v = threadIdx.x + i * nthr;
+            if (v < nvec) {
+                const uint4 yr = sy[v], zr = sy[nvec + v];
+                const T *ye = reinterpret_cast<const T *>(&yr);
+                const T *ze = reinterpret_cast<const T *>(&zr);
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    g[i][e] = to_f(ye[e]) * silu_ftz(to_f(ze[e]));
+                    ss = fmaf(g[i][e], g[i][e], ss);
+                }
+            }
+        }
+        // ---- CTA sum: red alternates between two halves, so one barrier per row suffices ----
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if ((threadIdx.x & 31) == 0) red[k & 1][threadIdx.x >> 5] = ss;
+        __syncthreads();
+        float tot = 0.f;
+        const float4 *red4 = reinterpret_cast<const float4 *>(red[k & 1]);
+        for (int i = 0; i < (nwarp4 >> 2); ++i) {
+            const float4 q = red4[i];
+            tot += (q.x + q.y) + (q.z + q.w);
+        }
+        const float rinv = rsqrtf(tot / (float)GS + eps);
+
+        // ---- scale and store ----
+        const float4 *w4 = reinterpret_cast<const float4 *>(w + (size_t)gi * GS);
+        uint4 *o4 = reinterpret_cast<uint4 *>(out + (size_t)t * C + (size_t)gi * GS);
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int v = threadIdx.x + i * nthr;
+            if (v < nvec) {
+                uint4 packed;
+                T *oe = reinterpret_cast<T *>(&packed);
+#pragma unroll
+                for (int q = 0; q < VEC / 4; ++q) {
+                    const float4 wv = __ldg(w4 + v * (VEC / 4) + q);
+                    oe[4 * q + 0] = from_f<T>(g[i][4 * q + 0] * rinv * wv.x);
+                    oe[4 * q + 1] = from_f<T>(g[i][4 * q + 1] * rinv * wv.y);
+                    oe[4 * q + 2] = from_f<T>(g[i][4 * q + 2] * rinv * wv.z);
+                    oe[4 * q + 3] = from_f<T>(g[i][4 * q + 3] * rinv * wv.w);
+                }
+                __stcs(o4 + v, packed);
+            }
+        }
+        t = tn;
+        gi = gn;
+        step(tn, gn);
+    }
+    allow_dependents();
+}
+
+template <typename T>
+static cudaError_t norm_stream_launch(const void *y, const void *z, const float *w, void *out, int T_rows, int C,
+                                      int n_groups, float eps, cudaStream_t st) {
+    constexpr auto kernel = gated_rmsnorm_stream_kernel<T>;
+    const int GS = C / n_groups;
+    const int threads = (GS / kNormStreamElems + (GS % kNormStreamElems ? 1 : 0) + 31) / 32 * 32;
+    const int smem = 2 * 2 * GS * (int)sizeof(T);
+    const int rows = T_rows * n_groups;  // below 2^30 (the dispatcher's rule), so r + gridDim.x fits
+    cudaError_t e = raise_smem_limit<kernel>(2 * 2 * kNormStreamRowBytes);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem)) != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    const long long resident = (long long)sms * per_sm;
+    const int grid = rows < resident ? rows : (int)resident;
+    return launch_pdl(kernel, dim3(grid), dim3(threads), smem, st, (const T *)y, (const T *)z, w, (T *)out, C, GS,
+                      n_groups, rows, eps);
+}
+
 template <typename T>
 static cudaError_t norm_launch(const void *y, const void *z, const float *w, void *out, int T_rows, int C,
                                int n_groups, float eps, cudaStream_t st) {
@@ -133,8 +313,15 @@ static cudaError_t norm_launch(const void *y, const void *z, const float *w, voi
 
 cudaError_t launch_gated_rmsnorm(int dtype, const void *y, const void *z, const float *w, void *out, int T_rows,
                                  int C, int n_groups, float eps, cudaStream_t st) {
-    if (dtype == SSD_DTYPE_BF16)
+    const int GS = C / n_groups;
+    const bool few_rows = (long long)T_rows * n_groups < (1ll << 30);
+    if (dtype == SSD_DTYPE_BF16) {
+        if (few_rows && GS * 2 <= kNormStreamRowBytes)
+            return norm_stream_launch<__nv_bfloat16>(y, z, w, out, T_rows, C, n_groups, eps, st);
         return norm_launch<__nv_bfloat16>(y, z, w, out, T_rows, C, n_groups, eps, st);
+    }
+    if (few_rows && GS * 4 <= kNormStreamRowBytes)
+        return norm_stream_launch<float>(y, z, w, out, T_rows, C, n_groups, eps, st);
     return norm_launch<float>(y, z, w, out, T_rows, C, n_groups, eps, st);
 }
 
