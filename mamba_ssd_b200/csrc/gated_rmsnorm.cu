@@ -28,6 +28,7 @@
 // result out.
 #include "common.cuh"
 #include "launch.h"
+#include "stream.cuh"
 #include "tc.cuh"
 
 namespace ssd {
@@ -135,26 +136,6 @@ constexpr int kNormStreamElems = 16;          // elements of a row per thread
 constexpr int kNormStreamRowBytes = 20480;    // largest y (or z) row of one group
 constexpr int kNormStreamMaxThreads = kNormStreamRowBytes / 2 / kNormStreamElems;  // bf16: 640
 
-__device__ __forceinline__ void cp_async16_first(void *smem, const void *gmem, uint64_t policy) {
-    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "l"(policy)
-                 : "memory");
-}
-// SiLU(z) = z / (1 + e^-z), with e^-z taken as 2^(-z log2 e) by the PTX approximate base-2
-// exponential and the division as a product with the approximate reciprocal, both in their
-// flush-to-zero forms (the build keeps denormals, and the non-flushing forms of those
-// instructions cost extra fix-up instructions per element).  Relative error about 2^-21;
-// a denormal z counts as zero.  -z is capped at 80 so that 1 + e^-z stays finite.
-__device__ __forceinline__ float silu_ftz(float z) {
-    float e, r;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(fminf(-z, 80.f) * 1.4426950408889634f));
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.f + e));
-    return z * r;
-}
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_prior() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-
 // rows: T_rows * n_groups (token-major, group fastest).  blockDim.x * VPT * VEC >= GS.
 template <typename T>
 __global__ void __launch_bounds__(kNormStreamMaxThreads) gated_rmsnorm_stream_kernel(
@@ -201,8 +182,8 @@ __global__ void __launch_bounds__(kNormStreamMaxThreads) gated_rmsnorm_stream_ke
             for (int i = 0; i < VPT; ++i) {
                 const int v = threadIdx.x + i * nthr;
                 if (v < nvec) {
-                    cp_async16_first(sy + v, y4 + v, first);
-                    cp_async16_first(sy + nvec + v, z4 + v, first);
+                    cp_async16(sy + v, y4 + v, first);
+                    cp_async16(sy + nvec + v, z4 + v, first);
                 }
             }
         }
@@ -217,7 +198,7 @@ __global__ void __launch_bounds__(kNormStreamMaxThreads) gated_rmsnorm_stream_ke
     request(r, t, gi, 0);
     for (int k = 0; r < rows; ++k, r += gridDim.x) {
         request(r + gridDim.x, tn, gn, (k + 1) & 1);
-        cp_async_wait_prior();  // every group but the newest: row r's copies have landed
+        cp_async_wait<1>();  // every group but the newest: row r's copies have landed
 
         // ---- gate and sum of squares (fp32), from the vectors this thread copied ----
         const uint4 *sy = ring_s + (size_t)(k & 1) * 2 * nvec;

@@ -68,6 +68,9 @@ def test_decode_steps_match_oracle(dtype, B, H, G, N, K):
     # 32-token strips and 8-token request batches: lengths around both, every K up to 8
     ("bf16", 2, 33, 64, 8), ("f32", 1, 65, 24, 5), ("bf16", 1, 31, 8, 6), ("bf16", 1, 32, 16, 7),
     ("f32", 2, 9, 32, 2),
+    # several 128-thread channel blocks with a partial last one, several sequences over several
+    # strips, odd K in bf16
+    ("bf16", 2, 100, 520, 5), ("bf16", 3, 70, 264, 3),
 ])
 def test_causal_conv_matches_oracle(dtype, B, L, Cc, K):
     rng = np.random.default_rng(L + Cc)
