@@ -1,4 +1,4 @@
-// stream.cuh -- helpers of the CUDA-core streaming kernels (the gated norm's streaming form):
+// stream.cuh -- helpers of the CUDA-core streaming kernels (the gated norm's streaming forms):
 // per-thread cp.async copies into a shared-memory ring, and a SiLU built on the flush-to-zero
 // approximate base-2 exponential and reciprocal.
 //

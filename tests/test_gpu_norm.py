@@ -1,8 +1,9 @@
 """GPU parity of ssd_gated_rmsnorm_fwd (through the C ABI) against the fp64 oracle.
 
 Shapes: the 2.7B-shaped block output (4096 tokens x 5120 channels, one norm group, and
-eight groups of 640), small ragged ones (8 channels, three groups of 8, 33 tokens), groups of
-1032 channels (the last thread of a row holds part of its 16 elements), both sides of the
+eight groups of 640), small ragged ones (8 channels, three groups of 8, 33 tokens), groups
+that the warp-per-row form takes with 1 to 4 vectors of 16 bytes per lane (up to 1024 bf16 /
+512 float32 channels, the largest rows it takes), groups of 1032 channels (the last thread of a row holds part of its 16 elements), both sides of the
 streaming form's limit (10240 bf16 / 5120 float32 channels per group streamed; 10248 / 5128
 staged), the largest group supported (32768 channels, past the default shared-memory limit),
 zero gates, eps = 0, and the empty call.  Tolerances are those of tests/parity.py ("norm").
@@ -35,6 +36,9 @@ def run(inp, n_groups, eps):
     ("f32", 33, 64, 2, 1e-6),
     ("bf16", 7, 8, 1, 1e-5),
     ("f32", 5, 24, 3, 0.0),
+    ("bf16", 64, 4096, 8, 1e-5),
+    ("bf16", 21, 3072, 3, 1e-5),
+    ("f32", 40, 1024, 2, 1e-5),
     ("bf16", 37, 2064, 2, 1e-5),
     ("f32", 19, 1032, 1, 1e-5),
     ("bf16", 9, 10240, 1, 1e-5),
