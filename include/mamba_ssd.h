@@ -363,7 +363,9 @@ SSD_API int ssd_causal_conv1d_fwd(const void *xBC, const void *conv_w, const voi
  *   w     [C]     float  per-channel scale
  *   out   [T, C]  dtype  must not overlap y or z
  *   n_groups             norm groups per token: C / n_groups consecutive channels each
- * The mean square is accumulated in float32.  Supported: C % n_groups == 0,
+ * The mean square is accumulated in float32; the gate's exponential and division and the
+ * reciprocal square root use the GPU's approximate instructions (relative error about 2^-21).
+ * Supported: C % n_groups == 0,
  * C / n_groups a multiple of 8 and at most 32768, n_groups <= 65535, eps >= 0 and finite.
  * Pointers 16-byte aligned.  Errors: SSD_ERR_INVALID_ARG (bad sizes, eps, dtype, pointers),
  * SSD_ERR_UNSUPPORTED (group size), SSD_ERR_CUDA.  T == 0 is a no-op.  Launched with
